@@ -1,0 +1,362 @@
+// C ABI of the AB-Attention hot path (declared in include/ab.h): argument
+// checks, workspace layout, TMA descriptors and kernel launches.  The library
+// allocates no memory; every buffer belongs to the caller.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "ab_attention.cuh"
+#include "ab_sample.cuh"
+#include "ab_select.cuh"
+
+namespace {
+
+using namespace ab;
+
+struct Dims {
+  int B, H, L, d, q_block, kv_block, C, iters;
+  int BH, Nq, Nkv, Kb;
+  float keep;
+  uint64_t seed;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int budget_of(int Nkv, double keep) {
+  double kb = std::floor(keep * double(Nkv) + 0.5);
+  if (kb < 1.0) kb = 1.0;
+  if (kb > double(Nkv)) kb = double(Nkv);
+  return int(kb);
+}
+
+// Host-side validation shared by every entry point.  `need_method` also checks
+// the fields only the sparse path uses.
+ab_status check_params(const ab_params* p, bool need_method, Dims* out) {
+  if (!p) return AB_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->L < 1 || p->L > (1 << 24)) return AB_ERR_INVALID_ARG;
+  if (int64_t(p->B) * p->H > (int64_t(1) << 20)) return AB_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return p->d > 0 ? AB_ERR_UNSUPPORTED : AB_ERR_INVALID_ARG;
+  if (p->q_block != 64 && p->q_block != 128) return p->q_block > 0 ? AB_ERR_UNSUPPORTED : AB_ERR_INVALID_ARG;
+  if (need_method) {
+    if (p->kv_block != 16 && p->kv_block != 32 && p->kv_block != 64)
+      return p->kv_block > 0 ? AB_ERR_UNSUPPORTED : AB_ERR_INVALID_ARG;
+    if (p->C != 1 && p->C != 2 && p->C != 4 && p->C != 8 && p->C != 16)
+      return (p->C >= 1 && p->C <= 16) ? AB_ERR_UNSUPPORTED : AB_ERR_INVALID_ARG;
+    if (p->kmeans_iters < 1 || p->kmeans_iters > 16) return AB_ERR_INVALID_ARG;
+    if (!(p->keep_ratio > 0.f) || !(p->keep_ratio <= 1.f)) return AB_ERR_INVALID_ARG;
+  }
+  Dims d{};
+  d.B = p->B; d.H = p->H; d.L = p->L; d.d = p->d; d.q_block = p->q_block;
+  d.kv_block = need_method ? p->kv_block : 16;
+  d.C = p->C; d.iters = p->kmeans_iters; d.keep = p->keep_ratio; d.seed = p->seed;
+  d.BH = p->B * p->H;
+  d.Nq = (p->L + d.q_block - 1) / d.q_block;
+  d.Nkv = (p->L + d.kv_block - 1) / d.kv_block;
+  d.Kb = need_method ? budget_of(d.Nkv, double(p->keep_ratio)) : 0;
+  if (int64_t(d.BH) * d.Nq > 0x7fffffff || int64_t(d.BH) * d.Nq * d.Nkv > (int64_t(1) << 40))
+    return AB_ERR_INVALID_ARG;
+  *out = d;
+  return AB_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Workspace {
+  size_t off_ksum, off_cent, off_cnt, total;
+};
+
+Workspace workspace_layout(const Dims& d) {
+  Workspace w{};
+  w.off_ksum = 0;
+  w.off_cent = align256(w.off_ksum + size_t(d.BH) * d.Nkv * d.d * 2);
+  w.off_cnt = align256(w.off_cent + size_t(d.BH) * d.Nq * d.C * d.d * 2);
+  w.total = align256(w.off_cnt + size_t(d.BH) * d.Nq * d.C * 4);
+  return w;
+}
+
+// ---------------------------------------------------------- TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor viewed as {inner, rows, outer}, 128B swizzle, box {64, box_rows, 1};
+// reads outside the tensor return zero.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {inner, rows, outer};
+  const cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+ab_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? AB_OK : AB_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- launches
+template <int D>
+ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, float* cent, int32_t* counts,
+                     uint8_t* ws, cudaStream_t st) {
+  const Workspace w = workspace_layout(d);
+  auto* ksum = reinterpret_cast<__nv_bfloat16*>(ws + w.off_ksum);
+  auto* cent_ws = reinterpret_cast<__nv_bfloat16*>(ws + w.off_cent);
+  auto* cnt_ws = reinterpret_cast<int32_t*>(ws + w.off_cnt);
+
+  // K-block summaries
+  {
+    const int64_t warps = int64_t(d.BH) * d.Nkv;
+    ksum_kernel<D><<<unsigned((warps + 7) / 8), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(K), ksum,
+                                                              d.BH, d.L, d.Nkv, d.kv_block);
+    if (launch_status() != AB_OK) return AB_ERR_CUDA;
+  }
+  // k-means per query block
+  {
+    CUtensorMap tmQ;
+    if (!make_map(&tmQ, Q, D, d.L, d.BH, 128)) return AB_ERR_CUDA;
+    const int smem = KmSmem<D>::kAlloc;
+    auto launch = [&](auto kern) -> ab_status {
+      if (set_smem(kern, smem) != cudaSuccess) return AB_ERR_CUDA;
+      kern<<<unsigned(d.BH * d.Nq), 128, smem, st>>>(tmQ, d.L, d.Nq, d.q_block, d.iters, cent, counts, cent_ws,
+                                                     cnt_ws);
+      return launch_status();
+    };
+    ab_status s;
+    switch (d.C) {
+      case 1: s = launch(kmeans_kernel<D, 1>); break;
+      case 2: s = launch(kmeans_kernel<D, 2>); break;
+      case 4: s = launch(kmeans_kernel<D, 4>); break;
+      case 8: s = launch(kmeans_kernel<D, 8>); break;
+      default: s = launch(kmeans_kernel<D, 16>); break;
+    }
+    if (s != AB_OK) return s;
+  }
+  // scores and block mass
+  {
+    CUtensorMap tmCent, tmKsum;
+    if (!make_map(&tmCent, cent_ws, D, uint64_t(d.BH) * d.Nq * d.C, 1, 128)) return AB_ERR_CUDA;
+    if (!make_map(&tmKsum, ksum, D, d.Nkv, d.BH, 256)) return AB_ERR_CUDA;
+    ScoreArgs a{};
+    a.L = d.L; a.Nq = d.Nq; a.Nkv = d.Nkv; a.q_block = d.q_block; a.kv_block = d.kv_block;
+    a.counts_ws = cnt_ws;
+    a.P = P;
+    a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
+    const int n_last = d.L - (d.Nkv - 1) * d.kv_block;
+    a.last_bias = float(std::log2(double(n_last) / double(d.kv_block)));
+    const int G = 128 / d.C;
+    const unsigned grid = unsigned(d.BH * ((d.Nq + G - 1) / G));
+    const int smem = ScSmem<D>::kAlloc;
+    auto launch = [&](auto kern) -> ab_status {
+      if (set_smem(kern, smem) != cudaSuccess) return AB_ERR_CUDA;
+      kern<<<grid, 160, smem, st>>>(tmCent, tmKsum, a);
+      return launch_status();
+    };
+    switch (d.C) {
+      case 1: return launch(score_kernel<D, 1>);
+      case 2: return launch(score_kernel<D, 2>);
+      case 4: return launch(score_kernel<D, 4>);
+      case 8: return launch(score_kernel<D, 8>);
+      default: return launch(score_kernel<D, 16>);
+    }
+  }
+}
+
+template <int D>
+ab_status run_attention(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* idx,
+                        const uint32_t* pi_q32, const int32_t* count, void* O, bool dense, cudaStream_t st) {
+  const int kvb = dense ? 128 : d.kv_block;
+  CUtensorMap tmQ, tmK, tmV;
+  if (!make_map(&tmQ, Q, D, d.L, d.BH, 128)) return AB_ERR_CUDA;
+  if (!make_map(&tmK, K, D, d.L, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
+  if (!make_map(&tmV, V, D, d.L, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
+  AttnArgs a{};
+  a.BH = d.BH; a.H = d.H; a.L = d.L; a.Nq = d.Nq; a.Nkv = dense ? (d.L + 127) / 128 : d.Nkv;
+  a.q_block = d.q_block;
+  a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
+  a.O = reinterpret_cast<__nv_bfloat16*>(O);
+  a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
+  const int smem = AttnSmem<D>::kAlloc;
+  auto launch = [&](auto kern) -> ab_status {
+    if (set_smem(kern, smem) != cudaSuccess) return AB_ERR_CUDA;
+    kern<<<unsigned(d.BH * d.Nq), 192, smem, st>>>(tmQ, tmK, tmV, a);
+    return launch_status();
+  };
+  switch (kvb) {
+    case 16: return launch(ab_attention_kernel<D, 16>);
+    case 32: return launch(ab_attention_kernel<D, 32>);
+    case 64: return launch(ab_attention_kernel<D, 64>);
+    default: return launch(ab_attention_kernel<D, 128>);
+  }
+}
+
+ab_status do_select(const Dims& d, const void* Q, const void* K, float* P, float* cent, int32_t* counts, void* ws,
+                    size_t ws_bytes, cudaStream_t st) {
+  if (!Q || !K || !P || !ws) return AB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(P) || !aligned16(ws)) return AB_ERR_INVALID_ARG;
+  if ((cent && !aligned16(cent)) || (counts && !aligned16(counts))) return AB_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_layout(d).total) return AB_ERR_WORKSPACE;
+  auto* w = reinterpret_cast<uint8_t*>(ws);
+  return d.d == 128 ? run_select<128>(d, Q, K, P, cent, counts, w, st) : run_select<64>(d, Q, K, P, cent, counts, w, st);
+}
+
+ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count, cudaStream_t st) {
+  if (!P || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
+  if (!aligned16(P) || !aligned16(idx) || !aligned16(pi_q32) || !aligned16(count)) return AB_ERR_INVALID_ARG;
+  SipArgs a{};
+  a.P = P; a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
+  a.H = d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
+  a.seed_lo = uint32_t(d.seed); a.seed_hi = uint32_t(d.seed >> 32);
+  sip_kernel<<<unsigned(d.BH * d.Nq), 256, 0, st>>>(a);
+  return launch_status();
+}
+
+ab_status do_attention(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* idx,
+                       const uint32_t* pi_q32, const int32_t* count, void* O, bool dense, cudaStream_t st) {
+  if (!Q || !K || !V || !O) return AB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return AB_ERR_INVALID_ARG;
+  if (!dense) {
+    if (!idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
+    if (!aligned16(idx) || !aligned16(pi_q32) || !aligned16(count)) return AB_ERR_INVALID_ARG;
+  }
+  return d.d == 128 ? run_attention<128>(d, Q, K, V, idx, pi_q32, count, O, dense, st)
+                    : run_attention<64>(d, Q, K, V, idx, pi_q32, count, O, dense, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t ab_budget(const ab_params* p) {
+  Dims d;
+  if (check_params(p, true, &d) != AB_OK) return -1;
+  return d.Kb;
+}
+
+ab_status ab_workspace_size(const ab_params* p, size_t* bytes) {
+  Dims d;
+  const ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  if (!bytes) return AB_ERR_INVALID_ARG;
+  *bytes = workspace_layout(d).total;
+  return AB_OK;
+}
+
+ab_status ab_select(const ab_params* p, const void* Q, const void* K, float* P, float* centroids, int32_t* counts,
+                    void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  const ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  return do_select(d, Q, K, P, centroids, counts, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,
+                    void* stream) {
+  Dims d;
+  const ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  return do_sample(d, P, idx, pi_q32, count, static_cast<cudaStream_t>(stream));
+}
+
+ab_status ab_attention(const ab_params* p, const void* Q, const void* K, const void* V, const int32_t* idx,
+                       const uint32_t* pi_q32, const int32_t* count, void* O, void* stream) {
+  Dims d;
+  const ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  return do_attention(d, Q, K, V, idx, pi_q32, count, O, false, static_cast<cudaStream_t>(stream));
+}
+
+ab_status ab_attention_dense(const ab_params* p, const void* Q, const void* K, const void* V, void* O,
+                             void* stream) {
+  Dims d;
+  const ab_status s = check_params(p, false, &d);
+  if (s != AB_OK) return s;
+  return do_attention(d, Q, K, V, nullptr, nullptr, nullptr, O, true, static_cast<cudaStream_t>(stream));
+}
+
+ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const void* V, float* P, int32_t* idx,
+                     uint32_t* pi_q32, int32_t* count, void* O, void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  if (!V || !O || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = do_select(d, Q, K, P, nullptr, nullptr, workspace, ws_bytes, st);
+  if (s != AB_OK) return s;
+  s = do_sample(d, P, idx, pi_q32, count, st);
+  if (s != AB_OK) return s;
+  return do_attention(d, Q, K, V, idx, pi_q32, count, O, false, st);
+}
+
+ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_host, const void* V_host,
+                          void* O_host, void* Q, void* K, void* V, float* P, int32_t* idx, uint32_t* pi_q32,
+                          int32_t* count, void* O, void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  if (!Q_host || !K_host || !V_host || !O_host || !Q || !K || !V || !O) return AB_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_layout(d).total) return AB_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = size_t(d.BH) * d.L * d.d * 2;
+  if (cudaMemcpyAsync(Q, Q_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
+  if (cudaMemcpyAsync(K, K_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
+  if (cudaMemcpyAsync(V, V_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
+  s = ab_forward(p, Q, K, V, P, idx, pi_q32, count, O, workspace, ws_bytes, stream);
+  if (s != AB_OK) return s;
+  if (cudaMemcpyAsync(O_host, O, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return AB_ERR_CUDA;
+  return AB_OK;
+}
+
+ab_status ab_get_device_error(void* stream, int32_t* code) {
+  if (!code) return AB_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (cudaMemcpyFromSymbolAsync(&host, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return AB_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return AB_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return AB_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return AB_ERR_CUDA;
+  *code = host;
+  return AB_OK;
+}
+
+const char* ab_status_string(ab_status s) {
+  switch (s) {
+    case AB_OK: return "ok";
+    case AB_ERR_INVALID_ARG: return "invalid argument";
+    case AB_ERR_UNSUPPORTED: return "unsupported size";
+    case AB_ERR_CUDA: return "CUDA error";
+    case AB_ERR_CAPACITY: return "list entry or count out of range";
+    case AB_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case AB_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

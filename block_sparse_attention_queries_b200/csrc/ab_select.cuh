@@ -1,0 +1,490 @@
+// IBCS, the intra-block clustering selector, for sm_100a.
+//
+// AB-Attention page ("AB-Attention: Video Difüzyon Transformer'larını
+// Hızlandırmak İçin Doğru Blok Dikkat Mekanizması"), section "AB-Attention ve
+// Üç Temel Yeniliği", IBCS item: the queries of each query block are clustered
+// in place (no token permutation) and the clusters estimate each KV block's
+// importance cheaply.  Three kernels:
+//
+//  ksum_kernel    kbar_j = mean of the valid keys of KV block j (bf16 out).
+//                 One warp per KV block; HBM-bound.
+//  kmeans_kernel  Lloyd k-means of one query block.  Distances come from
+//                 |mu_c|^2 - 2 q.mu_c with q.mu_c on the tensor cores (the
+//                 fp32 centroid split into bf16 hi + lo parts, two
+//                 accumulating MMAs, so the dot products keep ~16 bits);
+//                 argmin per query, then a deterministic ordered
+//                 per-cluster sum (ballot-ranked, ascending query order).
+//  score_kernel   S = mu kbar^T / sqrt(d) on the tensor cores for 128/C query
+//                 blocks at once (M = 128 centroid rows, N = 256 KV blocks per
+//                 chunk), per-centroid softmax over j in two passes (max and
+//                 sum, then normalised values), then the cluster-share mixture
+//                 P_ij = sum_c (n_c / n_i) p_cj reduced across the C lanes of
+//                 each query block with warp shuffles.
+#pragma once
+
+#include "ab_ptx.cuh"
+
+namespace ab {
+
+// ------------------------------------------------------------------- ksum
+template <int D>
+__global__ void __launch_bounds__(256) ksum_kernel(const __nv_bfloat16* __restrict__ K,
+                                                   __nv_bfloat16* __restrict__ Ksum, int BH, int L,
+                                                   int Nkv, int kv_block) {
+  constexpr int kPer = D / 32;  // dims per lane
+  const int warp_global = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (warp_global >= BH * Nkv) return;
+  const int bh = warp_global / Nkv;
+  const int j = warp_global - bh * Nkv;
+  const int n = min(kv_block, L - j * kv_block);
+  const __nv_bfloat16* src = K + (int64_t(bh) * L + int64_t(j) * kv_block) * D + lane * kPer;
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  for (int t = 0; t < n; ++t) {
+    if constexpr (kPer == 4) {
+      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src + int64_t(t) * D));
+      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+      acc[0] += __low2float(a);
+      acc[1] += __high2float(a);
+      acc[2] += __low2float(b);
+      acc[3] += __high2float(b);
+    } else {
+      const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(src + int64_t(t) * D));
+      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&raw);
+      acc[0] += __low2float(a);
+      acc[1] += __high2float(a);
+    }
+  }
+  const float inv = 1.f / float(n);
+  __nv_bfloat16* dst = Ksum + (int64_t(bh) * Nkv + j) * D + lane * kPer;
+  if constexpr (kPer == 4) {
+    uint2 out;
+    out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(dst) = out;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  }
+}
+
+// ----------------------------------------------------------------- k-means
+template <int D>
+struct KmSmem {
+  static constexpr int kSlabs = D / 64;
+  static constexpr int kOffQ = 0;                        // 128 x D bf16, SW128 slabs of 16 KB
+  static constexpr int kOffBhi = kOffQ + kSlabs * 16384; // 16 x D bf16, SW128 slabs of 2 KB
+  static constexpr int kOffBlo = kOffBhi + kSlabs * 2048;
+  static constexpr int kOffMu = kOffBlo + kSlabs * 2048; // fp32 [16][D]
+  static constexpr int kOffMusq = kOffMu + 16 * D * 4;   // fp32 [16]
+  static constexpr int kOffAssign = kOffMusq + 64;       // int [128]
+  static constexpr int kOffOrder = kOffAssign + 512;     // int [128]
+  static constexpr int kOffWcnt = kOffOrder + 512;       // int [4 warps][16]
+  static constexpr int kOffStart = kOffWcnt + 256;       // int [4][16] per-warp offsets + [17] starts
+  static constexpr int kOffBar = kOffStart + 256 + 128;
+  static constexpr int kOffMisc = kOffBar + 16;
+  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+// Element (row, e) of a 128B-swizzled K-major bf16 tile with 16 KB (or
+// `slab`-byte) slabs of 64 columns.
+__device__ __forceinline__ float sw_tile_get(const uint8_t* base, int slab_bytes, int row, int e) {
+  const int slab = e >> 6, col = e & 63;
+  const uint32_t off = uint32_t(slab * slab_bytes) + sw128_offset(uint32_t(row), uint32_t(col >> 3)) +
+                       uint32_t((col & 7) * 2);
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
+}
+
+// One CTA (128 threads) per query block.  Outputs: centroids (fp32, optional),
+// counts (optional), and for the scorer the bf16 centroids and int counts.
+template <int D, int C>
+__global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUtensorMap tmQ, int L, int Nq,
+                                                     int q_block, int iters, float* __restrict__ cent_out,
+                                                     int32_t* __restrict__ counts_out,
+                                                     __nv_bfloat16* __restrict__ cent_ws,
+                                                     int32_t* __restrict__ counts_ws) {
+  using SM = KmSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* mu = reinterpret_cast<float*>(smem + SM::kOffMu);
+  float* musq = reinterpret_cast<float*>(smem + SM::kOffMusq);
+  int* assign = reinterpret_cast<int*>(smem + SM::kOffAssign);
+  int* order = reinterpret_cast<int*>(smem + SM::kOffOrder);
+  int* wcnt = reinterpret_cast<int*>(smem + SM::kOffWcnt);    // [4][16]
+  int* woff = reinterpret_cast<int*>(smem + SM::kOffStart);   // [4][16]
+  int* cstart = woff + 64;                                    // [17]
+  const uint32_t bar_q = sbase + SM::kOffBar, bar_mma = sbase + SM::kOffBar + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kOffMisc + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x / Nq;
+  const int qi = blockIdx.x - bh * Nq;
+  const int n_i = min(q_block, L - qi * q_block);
+
+  if (tid == 0) {
+    mbar_init(bar_q, 1);
+    mbar_init(bar_mma, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_q, SM::kSlabs * 16384);
+    for (int s = 0; s < SM::kSlabs; ++s)
+      tma_load_3d(sbase + SM::kOffQ + s * 16384, &tmQ, bar_q, s * 64, qi * q_block, bh);
+  }
+  bool ok = mbar_wait(bar_q, 0, abort_flag);
+  ok = __syncthreads_and(ok);
+
+  const uint8_t* qtile = smem + SM::kOffQ;
+  // initial centroids: query at offset floor((c + 1/2) n_i / C); rows >= C are zero
+  for (int k = tid; k < 16 * D; k += 128) {
+    const int c = k / D, e = k - c * D;
+    float v = 0.f;
+    if (c < C) {
+      const int src = ((2 * c + 1) * n_i) / (2 * C);
+      v = sw_tile_get(qtile, 16384, src, e);
+    }
+    mu[k] = v;
+  }
+  __syncthreads();
+
+  const uint32_t idesc = idesc_bf16_f32(128, 16, 0, 0);
+  for (int it = 0; it < iters && ok; ++it) {
+    // centroid tiles (bf16 hi and lo parts, 16 rows, K-major SW128) and |mu|^2
+    for (int k = tid; k < 16 * (D / 8); k += 128) {
+      const int c = k / (D / 8), ch = k - c * (D / 8);  // 8-element chunk
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float v0 = mu[c * D + ch * 8 + 2 * h], v1 = mu[c * D + ch * 8 + 2 * h + 1];
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
+        hi[h] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+        lo[h] = pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+      }
+      const uint32_t off = uint32_t((ch >> 3) * 2048) + sw128_offset(uint32_t(c), uint32_t(ch & 7));
+      *reinterpret_cast<uint4*>(smem + SM::kOffBhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(smem + SM::kOffBlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    if (warp == 0) {
+      for (int c = 0; c < C; ++c) {
+        float s = 0.f;
+        for (int e = lane; e < D; e += 32) s = fmaf(mu[c * D + e], mu[c * D + e], s);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) musq[c] = s;
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+        const uint32_t boff = (kk >> 2) * 2048 + (kk & 3) * 32;
+        mma_bf16_ss(tmem, smem_desc_sw128(sbase + SM::kOffQ + aoff, 16, 1024),
+                    smem_desc_sw128(sbase + SM::kOffBhi + boff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem, smem_desc_sw128(sbase + SM::kOffQ + aoff, 16, 1024),
+                    smem_desc_sw128(sbase + SM::kOffBlo + boff, 16, 1024), idesc, 1u);
+      }
+      mma_commit(bar_mma);
+    }
+    ok = mbar_wait(bar_mma, it & 1, abort_flag);
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    tc_fence_after();
+    // dot products of this thread's query with the 16 centroid rows
+    uint32_t dv[32];
+    tmem_ld32(tmem + (uint32_t(warp * 32) << 16), dv);
+    tmem_wait_ld();
+    int best = C;  // C marks "no query" (rows beyond the block)
+    if (tid < n_i) {
+      float bd = INFINITY;
+      best = 0;
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        const float dist = fmaf(-2.f, __uint_as_float(dv[c]), musq[c]);
+        if (dist < bd) {  // strict: ties go to the lower c
+          bd = dist;
+          best = c;
+        }
+      }
+    }
+    assign[tid] = best;
+    // ordered bucket of each query: warp ballots give the rank inside the warp
+    int my_rank = 0;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, best == c);
+      if (best == c) my_rank = __popc(bal & ((1u << lane) - 1u));
+      if (lane == 0) wcnt[warp * 16 + c] = __popc(bal);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0;
+      for (int c = 0; c < C; ++c) {
+        cstart[c] = run;
+        for (int w = 0; w < 4; ++w) {
+          woff[w * 16 + c] = run;
+          run += wcnt[w * 16 + c];
+        }
+      }
+      cstart[C] = run;
+    }
+    __syncthreads();
+    if (best < C) order[woff[warp * 16 + best] + my_rank] = tid;
+    __syncthreads();
+    // new centroid = mean of the members, summed in ascending query order
+    for (int e = tid; e < D; e += 128) {
+      for (int c = 0; c < C; ++c) {
+        const int b0 = cstart[c], b1 = cstart[c + 1];
+        if (b1 == b0) continue;  // empty cluster keeps its centroid
+        float s = 0.f;
+        for (int k = b0; k < b1; ++k) s += sw_tile_get(qtile, 16384, order[k], e);
+        mu[c * D + e] = s / float(b1 - b0);
+      }
+    }
+    __syncthreads();
+  }
+
+  if (ok) {
+    const int64_t row0 = (int64_t(bh) * Nq + qi) * C;
+    for (int k = tid; k < C * D; k += 128) {
+      const float v = mu[k];
+      if (cent_out) cent_out[row0 * D + k] = v;
+      cent_ws[row0 * D + k] = __float2bfloat16_rn(v);
+    }
+    if (tid < C) {
+      const int n_c = cstart[tid + 1] - cstart[tid];
+      if (counts_out) counts_out[row0 + tid] = n_c;
+      counts_ws[row0 + tid] = n_c;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+}
+
+// ------------------------------------------------------------------ scores
+template <int D>
+struct ScSmem {
+  static constexpr int kSlabs = D / 64;
+  static constexpr int kA = kSlabs * 16384;          // 128 x D bf16
+  static constexpr int kB = kSlabs * 32768;          // 256 x D bf16
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kA;           // 2 stages
+  static constexpr int kOffW = kOffB + 2 * kB;       // float [128] row weights
+  static constexpr int kOffBar = kOffW + 512;        // a_full, b_full[2], b_empty[2], s_full[2], t_free[2]
+  static constexpr int kOffMisc = kOffBar + 10 * 8;
+  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+struct ScoreArgs {
+  int L, Nq, Nkv, q_block, kv_block;
+  const int32_t* counts_ws;  // [BH, Nq, C]
+  float* P;                  // [BH, Nq, Nkv]
+  float scale_log2;          // log2(e) / sqrt(d)
+  float last_bias;           // log2(n_last / kv_block) of the last KV block
+};
+
+// Reduce 32 per-lane values over aligned groups of C lanes and scatter the
+// sums: after the call lane g (g = lane % C) of a group holds, in v[0 ..
+// 32/C), the group sums of columns [g * 32/C, (g + 1) * 32/C).
+template <int C>
+__device__ __forceinline__ void group_reduce_scatter(float (&v)[32], int lane) {
+#pragma unroll
+  for (int m = C / 2; m >= 1; m >>= 1) {
+    const bool upper = (lane & m) != 0;
+    const int half = 32 * m / C;  // values still held per lane, halved by this stage
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (k < half) {
+        const float send = upper ? v[k] : v[k + half];
+        const float keep = upper ? v[k + half] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+      }
+    }
+  }
+}
+
+template <int D, int C>
+__global__ void __launch_bounds__(160, 1)
+    score_kernel(const __grid_constant__ CUtensorMap tmCent, const __grid_constant__ CUtensorMap tmKsum,
+                 const ScoreArgs a) {
+  using SM = ScSmem<D>;
+  constexpr int G = 128 / C;  // query blocks per CTA
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + SM::kOffBar;
+  auto bar = [&](int k) { return bar0 + 8u * uint32_t(k); };
+  enum { kA = 0, kBFull = 1, kBEmpty = 3, kSFull = 5, kTFree = 7, kDrain = 9 };
+  float* roww = reinterpret_cast<float*>(smem + SM::kOffW);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kOffMisc + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int groups_per_head = (a.Nq + G - 1) / G;
+  const int bh = blockIdx.x / groups_per_head;
+  const int i0 = (blockIdx.x - bh * groups_per_head) * G;
+  const int nchunks = (a.Nkv + 255) / 256;
+
+  if (tid == 0) {
+    mbar_init(bar(kA), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBFull + s), 1);
+      mbar_init(bar(kBEmpty + s), 1);
+      mbar_init(bar(kSFull + s), 1);
+      mbar_init(bar(kTFree + s), 128);
+    }
+    mbar_init(bar(kDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (tid < 128) {
+    // row r = (query block i0 + r / C, centroid r % C): weight n_c / n_i (0 if none)
+    const int i = i0 + tid / C;
+    float w = 0.f;
+    if (tid < G * C && i < a.Nq) {
+      const int n_i = min(a.q_block, a.L - i * a.q_block);
+      w = float(a.counts_ws[(int64_t(bh) * a.Nq + i) * C + (tid % C)]) / float(n_i);
+    }
+    roww[tid] = w;
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = 2 * nchunks;  // pass 0: max and sum; pass 1: values
+
+  if (warp == 4) {
+    if (lane == 0) {
+      bool ok = true;
+      mbar_arrive_expect_tx(bar(kA), SM::kA);
+      for (int s = 0; s < SM::kSlabs; ++s)
+        tma_load_3d(sbase + SM::kOffA + s * 16384, &tmCent, bar(kA), s * 64, (bh * a.Nq + i0) * C, 0);
+      auto load_b = [&](int g) {
+        const int st = g & 1;
+        const int chunk = g % nchunks;
+        mbar_arrive_expect_tx(bar(kBFull + st), SM::kB);
+        for (int s = 0; s < SM::kSlabs; ++s)
+          tma_load_3d(sbase + SM::kOffB + st * SM::kB + s * 32768, &tmKsum, bar(kBFull + st), s * 64,
+                      chunk * 256, bh);
+      };
+      load_b(0);
+      if (total > 1) load_b(1);
+      ok = mbar_wait(bar(kA), 0, abort_flag);
+      const uint32_t idesc = idesc_bf16_f32(128, 256, 0, 0);
+      for (int g = 0; g < total && ok; ++g) {
+        const int st = g & 1;
+        if (!mbar_wait(bar(kBFull + st), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (g >= 2 && !mbar_wait(bar(kTFree + st), ((g - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * 32768 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + uint32_t(st * 256), smem_desc_sw128(sbase + SM::kOffA + aoff, 16, 1024),
+                      smem_desc_sw128(sbase + SM::kOffB + st * SM::kB + boff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(kSFull + st));
+        mma_commit(bar(kBEmpty + st));
+        if (g + 2 < total) {
+          if (!mbar_wait(bar(kBEmpty + st), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+          load_b(g + 2);
+        }
+      }
+      mma_commit(bar(kDrain));
+      mbar_wait_drain(bar(kDrain), 0);
+    }
+  } else {
+    const int r = tid;  // centroid row == TMEM lane
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const float w = roww[r];
+    float M = -INFINITY, Z = 0.f;
+    bool ok = true;
+    for (int g = 0; g < total && ok; ++g) {
+      const int st = g & 1;
+      const int chunk = g % nchunks;
+      const bool pass2 = g >= nchunks;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + st), (g >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const float inv_z = pass2 ? w / Z : 0.f;
+#pragma unroll 1
+      for (int piece = 0; piece < 8; ++piece) {
+        uint32_t raw[32];
+        tmem_ld32(tmem + lane_base + uint32_t(st * 256 + piece * 32), raw);
+        tmem_wait_ld();
+        const int j0 = chunk * 256 + piece * 32;
+        float v[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const int j = j0 + k;
+          float x = __uint_as_float(raw[k]) * a.scale_log2;
+          if (j == a.Nkv - 1) x += a.last_bias;
+          v[k] = (j < a.Nkv) ? x : -INFINITY;
+        }
+        if (!pass2) {
+          float pm = M;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) pm = fmaxf(pm, v[k]);
+          float s = 0.f;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) s += ex2_approx(v[k] - pm);
+          Z = Z * ex2_approx(M - pm) + s;  // M = -inf on the first piece: factor 0
+          M = pm;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = ex2_approx(v[k] - M) * inv_z;
+          group_reduce_scatter<C>(v, lane);
+          constexpr int kPer = 32 / C;
+          const int gl = lane % C;
+          const int i = i0 + r / C;
+          if (i < a.Nq && (r / C) < G) {
+            float* prow = a.P + (int64_t(bh) * a.Nq + i) * a.Nkv;
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+              const int j = j0 + gl * kPer + k;
+              if (j < a.Nkv) prow[j] = v[k];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kTFree + st));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace ab

@@ -1,0 +1,203 @@
+/*
+ * ab.h -- C ABI of the AB-Attention (Accurate Block Attention) hot path for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is the one summarised on the page "AB-Attention: Video Difüzyon
+ * Transformer'larını Hızlandırmak İçin Doğru Blok Dikkat Mekanizması"
+ * (Edumints summary of Hugging Face Papers entry 2610.39663), called "the
+ * AB-Attention page" below.  Its section "AB-Attention ve Üç Temel Yeniliği"
+ * names three parts, each behind one call here:
+ *
+ *   ab_select     IBCS, the intra-block clustering selector: cluster the queries
+ *                 inside each query block (no token permutation) and estimate
+ *                 every KV block's share of the block's attention mass.
+ *   ab_sample     SIP, sampling with inclusion-probability weighting: draw KV
+ *                 blocks in proportion to that estimate and keep each kept
+ *                 block's inverse inclusion probability.
+ *   ab_attention  the kernel that packs the small kept KV blocks into full
+ *                 tensor-core tiles and computes the 1/pi-weighted softmax, an
+ *                 estimate of softmax(Q K^T / sqrt(d)) V (the formula of the
+ *                 "Cross-Attention (Çapraz Dikkat Mekanizması)" glossary page,
+ *                 "Cross-Attention Nasıl Çalışır?").
+ *
+ * ab_attention_dense computes exact dense attention with the same kernel
+ * family (the reference point for speed), ab_forward runs the three steps on
+ * device buffers, ab_forward_host runs them on host buffers.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors Q, K, V, O are [B, H, L, d] bfloat16, contiguous, d fastest,
+ *    tokens in raster order of the (t, y, x) grid.  Query blocks are the
+ *    contiguous runs of q_block tokens (Nq = ceil(L / q_block)); KV blocks
+ *    the runs of kv_block tokens (Nkv = ceil(L / kv_block)); the last block of
+ *    each kind may be partial.
+ *  - Memory: the caller allocates and owns every buffer (device memory unless a
+ *    call says "host"); the library allocates nothing and frees nothing.
+ *    Every device pointer must be 16-byte aligned.
+ *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *    Every call only enqueues work on it and returns; results are ready when
+ *    the stream reaches them.  The library keeps no state between calls other
+ *    than the device error word.
+ *  - Errors: arguments are checked on the host before anything is launched;
+ *    a bad argument returns AB_ERR_INVALID_ARG (or AB_ERR_UNSUPPORTED for a
+ *    valid but unimplemented size) and enqueues nothing.  AB_ERR_CUDA reports
+ *    a failed launch.  Problems found on the device (a list entry out of range,
+ *    a count above capacity, a pipeline wait that timed out) never trap: the
+ *    kernel records the first one in the device error word and skips the bad
+ *    work; read it with ab_get_device_error.
+ *  - Randomness: the only random numbers are SIP's draws, from
+ *    Philox4x32-10 (Salmon et al., SC'11) keyed by ab_params.seed, so a call
+ *    is deterministic for fixed inputs and seed.
+ */
+#ifndef AB_ATTENTION_AB_H_
+#define AB_ATTENTION_AB_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  AB_OK = 0,
+  AB_ERR_INVALID_ARG = 1, /* null/misaligned pointer, size out of range */
+  AB_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. d = 96) */
+  AB_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  AB_ERR_CAPACITY = 4,    /* device: count > Nkv or a list index >= Nkv */
+  AB_ERR_TIMEOUT = 5,     /* device: a pipeline wait gave up (kernel ended early) */
+  AB_ERR_WORKSPACE = 6,   /* workspace too small */
+} ab_status;
+
+/* Problem description shared by every call. */
+typedef struct {
+  int32_t B, H, L, d;        /* batch, heads, tokens, head dim; d in {64, 128}; 1 <= L <= 2^24 */
+  int32_t q_block;           /* query block size, 64 or 128 */
+  int32_t kv_block;          /* KV block size, 16, 32 or 64 */
+  int32_t C;                 /* clusters per query block: 1, 2, 4, 8 or 16 */
+  int32_t kmeans_iters;      /* Lloyd iterations, 1..16 (3 in the workloads) */
+  float keep_ratio;          /* target kept fraction of KV blocks, in (0, 1] */
+  uint64_t seed;             /* Philox key of the SIP draws */
+} ab_params;
+
+/*
+ * Kept KV blocks per query block in expectation:
+ *   Kb = clamp(floor(keep_ratio * Nkv + 1/2), 1, Nkv)   (computed in double).
+ * Returns -1 if p is invalid.
+ */
+int32_t ab_budget(const ab_params* p);
+
+/* Bytes of device workspace ab_select (and ab_forward) need for *p. */
+ab_status ab_workspace_size(const ab_params* p, size_t* bytes);
+
+/*
+ * IBCS (AB-Attention page, "AB-Attention ve Üç Temel Yeniliği", IBCS item).
+ * For every (b, h) and query block i:
+ *   kbar_j  = mean of the valid keys of KV block j;
+ *   mu, n_c = Lloyd k-means of the block's n_i queries with C clusters and
+ *             kmeans_iters iterations (initial centroid c is the query at
+ *             offset floor((c + 1/2) n_i / C); an empty cluster keeps its
+ *             centroid; n_c are the sizes of the last assignment);
+ *   S_cj    = mu_c . kbar_j / sqrt(d) + ln n_j   (n_j = valid keys in block j);
+ *   P[i,j]  = sum_c (n_c / n_i) softmax_j(S_cj).
+ * The centroid-summary product runs on the tensor cores in bfloat16 with fp32
+ * accumulation, so P matches an exact evaluation to a few 1e-3 relative.
+ *
+ *   Q, K       device, [B, H, L, d] bf16.
+ *   P          device, out, [B, H, Nq, Nkv] fp32; each row sums to 1.
+ *   centroids  device, out, optional (NULL), [B, H, Nq, C, d] fp32.
+ *   counts     device, out, optional (NULL), [B, H, Nq, C] int32.
+ *   workspace  device scratch of at least ab_workspace_size bytes
+ *              (AB_ERR_WORKSPACE otherwise); contents need no initialisation.
+ */
+ab_status ab_select(const ab_params* p, const void* Q, const void* K, float* P, float* centroids,
+                    int32_t* counts, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * SIP (AB-Attention page, "AB-Attention ve Üç Temel Yeniliği", SIP item).
+ * For every row (b, h, i) of P, entirely in integer arithmetic:
+ *   W_j  = max(1, floor(P[i,j] * 2^24));
+ *   inclusion probabilities proportional to W, capped at 1, summing to Kb: the
+ *   capped set A grows until stable by adding every j not in A with
+ *   R W_j >= S (R = Kb - |A|, S = sum of W_j over j not in A); then
+ *   Pi_j = 2^32 for j in A, else max(1, floor(R W_j 2^32 / S)); pi_j = Pi_j / 2^32;
+ *   u_j  = word (j mod 4) of Philox4x32-10(counter (j div 4, i, h, b),
+ *          key (seed mod 2^32, seed div 2^32)); block j is kept iff u_j < Pi_j.
+ * Kept blocks are written in ascending j order.
+ *
+ *   P       device, [B, H, Nq, Nkv] fp32 (any source).
+ *   idx     device, out, [B, H, Nq, Nkv] int32: row r's first count[r]
+ *           entries are the kept j; the rest are left untouched.
+ *   pi_q32  device, out, [B, H, Nq, Nkv] uint32: Pi_j mod 2^32 of each kept
+ *           block (0 encodes pi = 1), aligned with idx.
+ *   count   device, out, [B, H, Nq] int32.
+ * Results are bit-identical to the integer specification above.
+ */
+ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,
+                    void* stream);
+
+/*
+ * 1/pi-weighted block-sparse attention (AB-Attention page, SIP item: one pass
+ * estimates dense attention instead of truncating it; "Donanım Dostu Çekirdek"
+ * item: KV blocks much smaller than a tile are packed into full tensor-core
+ * tiles).  For query q of block i, with s_k = q . k / sqrt(d) and
+ * w_j = 2^32 / Pi_j (1 when pi_q32 = 0):
+ *   O_q = sum_{j in list(i)} w_j sum_{k in j, k < L} e^{s_k} v_k
+ *       / sum_{j in list(i)} w_j sum_{k in j, k < L} e^{s_k};
+ * a query block with count 0 gets O = 0.  The lists may come from ab_sample
+ * or from any other source; they must be ascending or not, but each entry must
+ * satisfy 0 <= idx < Nkv and count <= Nkv (violations raise AB_ERR_CAPACITY on
+ * the device and the offending entries or rows are skipped).
+ *
+ *   Q, K, V  device, [B, H, L, d] bf16.
+ *   idx, pi_q32, count  device, as written by ab_sample.
+ *   O        device, out, [B, H, L, d] bf16 (round to nearest even).
+ */
+ab_status ab_attention(const ab_params* p, const void* Q, const void* K, const void* V, const int32_t* idx,
+                       const uint32_t* pi_q32, const int32_t* count, void* O, void* stream);
+
+/*
+ * Dense attention O = softmax(Q K^T / sqrt(d)) V, bidirectional, no mask
+ * (Cross-Attention glossary page, "Cross-Attention Nasıl Çalışır?"; the
+ * AB-Attention page's "3D tam dikkat").  Uses q_block (64 or 128), B, H, L, d
+ * from *p; the other fields are ignored.  Same layout rules as ab_attention.
+ */
+ab_status ab_attention_dense(const ab_params* p, const void* Q, const void* K, const void* V, void* O,
+                             void* stream);
+
+/*
+ * The three steps in order on device buffers: ab_select (into P, with
+ * centroids/counts not kept), ab_sample, ab_attention.  `workspace` as for
+ * ab_select.
+ */
+ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const void* V, float* P,
+                     int32_t* idx, uint32_t* pi_q32, int32_t* count, void* O, void* workspace,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * ab_forward from HOST buffers: copies Q_host, K_host, V_host (host, [B, H, L,
+ * d] bf16; page-locked memory gives asynchronous copies) to the device buffers
+ * Q, K, V, runs ab_forward, and copies O back to O_host (host, [B, H, L, d]
+ * bf16).  All copies are enqueued on `stream`; O_host is valid once the stream
+ * has been synchronised.  The device buffers are owned by the caller.
+ */
+ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_host, const void* V_host,
+                          void* O_host, void* Q, void* K, void* V, float* P, int32_t* idx,
+                          uint32_t* pi_q32, int32_t* count, void* O, void* workspace, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * Reads and clears the device error word of the current device, after
+ * synchronising `stream`.  *code receives AB_OK or the first ab_status raised
+ * on the device since the last read.  Returns AB_ERR_CUDA if the read failed.
+ */
+ab_status ab_get_device_error(void* stream, int32_t* code);
+
+/* Static description of a status code. */
+const char* ab_status_string(ab_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AB_ATTENTION_AB_H_ */

@@ -1,0 +1,77 @@
+"""The C ABI library loads on a machine without a GPU, exports every function
+include/ab.h declares, and rejects bad arguments on the host before any CUDA
+call (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_queries_b200 as ab
+from block_sparse_attention_queries_b200 import build as abbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    abbuild.build()
+    return ab.lib()
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "ab.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(ab_\w+)\s*\(", txt, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert set(declared) == set(ab.EXPORTS), declared
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_budget_and_workspace(lib):
+    p = ab.Params(B=1, H=40, L=32760, d=128, q_block=128, kv_block=16, C=8, keep_ratio=0.11)
+    assert ab.budget(p) == 225
+    assert ab.budget(ab.Params(B=1, H=24, L=118800, d=128, keep_ratio=0.08)) == 594
+    assert ab.budget(ab.Params(B=1, H=1, L=1024, d=64, q_block=64, C=4, keep_ratio=0.10)) == 6
+    ws = ab.workspace_size(p)
+    # K summaries + bf16 centroids + counts
+    assert ws >= 40 * 2048 * 128 * 2 + 40 * 256 * 8 * 128 * 2 + 40 * 256 * 8 * 4
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("d", 96, 2), ("d", 0, 1), ("q_block", 32, 2), ("kv_block", 8, 2), ("kv_block", 0, 1),
+    ("C", 3, 2), ("C", 0, 1), ("C", 17, 1), ("kmeans_iters", 0, 1), ("keep_ratio", 0.0, 1),
+    ("keep_ratio", 1.5, 1), ("L", 0, 1), ("B", 0, 1), ("L", 2**24 + 1, 1),
+])
+def test_invalid_params_rejected_on_host(lib, field, value, status):
+    kw = dict(B=1, H=2, L=1000, d=128, q_block=128, kv_block=16, C=8, keep_ratio=0.1)
+    kw[field] = value
+    p = ab.Params(**kw).c()
+    n = ctypes.c_size_t(0)
+    assert lib.ab_workspace_size(ctypes.byref(p), ctypes.byref(n)) == status
+    assert lib.ab_budget(ctypes.byref(p)) == -1
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    p = ab.Params(B=1, H=1, L=256, d=64, q_block=64, kv_block=16, C=4).c()
+    # null pointers
+    assert lib.ab_select(ctypes.byref(p), None, None, None, None, None, None, 0, None) == 1
+    assert lib.ab_sample(ctypes.byref(p), None, None, None, None, None) == 1
+    assert lib.ab_attention(ctypes.byref(p), None, None, None, None, None, None, None, None) == 1
+    assert lib.ab_attention_dense(ctypes.byref(p), None, None, None, None, None) == 1
+    # misaligned (never dereferenced: rejected before any launch)
+    bad = ctypes.c_void_p(0x1000 + 8)
+    good = ctypes.c_void_p(0x1000)
+    assert lib.ab_attention_dense(ctypes.byref(p), bad, good, good, good, None) == 1
+    # workspace too small
+    assert lib.ab_select(ctypes.byref(p), good, good, good, None, None, good, 16, None) == 6
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.ab_status_string(s)
+    assert ab.status_string(6) == "workspace too small"
