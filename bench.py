@@ -1,0 +1,405 @@
+"""Benchmark of the AB-Attention hot path on B200: one attention layer of the
+Wan2.1-14B-shaped 480p workload (B=1, H=40, 21x30x52 = 32760 tokens, d=128,
+query block 128, KV block 16, C=8, 11% of KV blocks kept).
+
+A step is one pass of the whole path: ab_select (IBCS) -> ab_sample (SIP)
+-> ab_attention (packed 1/pi-weighted sparse attention) over one layer's
+Q, K, V.  Inputs are synthetic (seeded Fourier-feature Q/K, Gaussian V with
+outlier tokens) at the workload's shapes; each of Q, K, V is 335 MB, larger
+than the 126 MB L2, so no explicit L2 flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  The metric is dense-equivalent attention
+TFLOP/s (4 B H L^2 d flop per layer / time per layer).  `--impl reference`
+times the CPU oracle (the reference arm of this repository) on a bounded
+sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "dense-equivalent attention TFLOPS/s + tensor-pipe util; ms per attention layer"
+UNIT = "TFLOP/s"
+WORKLOAD = "wan2.1-14b-480p-self-attention"
+
+
+def workload():
+    from block_sparse_attention_queries_b200.synthetic import WORKLOADS
+    return WORKLOADS["wan480"]
+
+
+def dense_flop(w) -> float:
+    return 4.0 * w.B * w.H * float(w.L) ** 2 * w.d
+
+
+def config_dict(w, extra=None):
+    c = {"workload": WORKLOAD, "B": w.B, "H": w.H, "grid_txy": list(w.grid), "L": w.L, "d": w.d,
+         "q_block": w.q_block, "kv_block": w.kv_block, "C": w.C, "kmeans_iters": w.kmeans_iters,
+         "keep_ratio": w.keep_ratio, "sampler_seed": 42, "data_seed": 1234,
+         "l2": "inputs larger than L2 (Q, K, V 335 MB each); no flush"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def peaks():
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), float(pk["hbm_gbs"]), "measured (burst)"
+    except Exception:
+        return 1590.0, 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            import torch
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id if hasattr(
+                torch.cuda.get_device_properties(device_index), "pci_bus_id") else None
+        except Exception:
+            bus = None
+        self.id = bus if bus else str(device_index)
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.id}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def wait_first_sample(self, timeout_s: float = 5.0):
+        t = time.time()
+        while self.proc is not None and time.time() - t < timeout_s:
+            if os.path.getsize(self.path) > 0:
+                return
+            time.sleep(0.05)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 7:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[3 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------- our arm (GPU)
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import block_sparse_attention_queries_b200 as ab
+    from block_sparse_attention_queries_b200.synthetic import make_workload_qkv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", rank=rank, world_size=world, device_id=dev,
+                                timeout=datetime.timedelta(seconds=120))
+
+    w = workload()
+    p = ab.Params.of(w, seed=42)
+    # weak scaling: every rank runs its own layer (independent batch element)
+    Qc, Kc, Vc = make_workload_qkv(w, seed=1234 + rank)
+    Q, K, V = (t.to(dev) for t in (Qc, Kc, Vc))
+    bufs = ab.Buffers(p, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        _select(ab, p, Q, K, bufs)
+        if ev is not None:
+            ev[1].record(stream)
+        _sample(ab, p, bufs)
+        if ev is not None:
+            ev[2].record(stream)
+        ab.ab_attention(p, Q, K, V, bufs.idx, bufs.pi_q32, bufs.count, out=bufs.O)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    code = ab.device_error(dev)
+    if code:
+        raise SystemExit(f"device error during warm-up: {ab.status_string(code)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()  # nvidia-smi needs a moment before its first sample
+    clocks.wait_first_sample()
+    barrier()
+    t0.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    sel_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    smp_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    att_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    code = ab.device_error(dev)
+    if code:
+        raise SystemExit(f"device error in the timed region: {ab.status_string(code)}")
+
+    # executed algorithmic attention flop from the last step's lists: 4 d sum_i n_i sum_{j in S_i} n_j
+    cnt = bufs.count.cpu().numpy().astype(np.int64)
+    idx = bufs.idx.cpu().numpy()
+    n_last = w.L - (w.Nkv - 1) * w.kv_block
+    last_kept = sum(int((idx[0, h, i, :cnt[0, h, i]] == w.Nkv - 1).any())
+                    for h in range(w.H) for i in range(w.Nq) if cnt[0, h, i] > 0)
+    n_i = np.array([min(w.q_block, w.L - i * w.q_block) for i in range(w.Nq)], np.int64)
+    keys = cnt * w.kv_block
+    exec_flop = 4.0 * w.d * float((n_i[None, None, :] * keys).sum())
+    # correct the (at most one per row) partial last KV block
+    if last_kept:
+        part = np.zeros_like(cnt)
+        for h in range(w.H):
+            for i in range(w.Nq):
+                c = cnt[0, h, i]
+                if c and (idx[0, h, i, :c] == w.Nkv - 1).any():
+                    part[0, h, i] = w.kv_block - n_last
+        exec_flop -= 4.0 * w.d * float((n_i[None, None, :] * part).sum())
+    kept_frac = float(cnt.sum()) / (w.B * w.H * w.Nq * w.Nkv)
+
+    # max over ranks
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    ms_step = total_ms / args.steps
+    value = dense_flop(w) * world / (ms_step * 1e-3) / 1e12
+    att_avg = statistics.mean(att_ms)
+    bf16_peak, hbm_peak, peak_kind = peaks()
+    achieved = exec_flop / (att_avg * 1e-3) / 1e12
+
+    out = None
+    if rank == 0:
+        # e2e through the public C ABI with host buffers (copies inside the region)
+        e2e = run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, max(2, min(args.steps, 5)))
+        dense_ms = run_dense(ab, p, Q, K, V, dev, 3)
+        cpu = cpu_baseline(w, args)
+        out = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(w, {"parallelism": f"dp{world} (independent layers per GPU)"}),
+            "ms_per_layer": round(ms_step, 4),
+            "ms_select": round(statistics.mean(sel_ms), 4), "ms_sample": round(statistics.mean(smp_ms), 4),
+            "ms_attention": round(att_avg, 4),
+            "executed_tflops_attention": round(achieved, 2),
+            "kept_block_fraction": round(kept_frac, 5),
+            "dense_kernel_ms": round(dense_ms, 3),
+            "speedup_vs_own_dense_kernel": round(dense_ms / ms_step, 3),
+            "gpu_launches": 5 * args.steps,
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / bf16_peak, 4), "traffic": None,
+                         "kernel": "ab_attention_kernel<128,16>", "peak_kind": peak_kind,
+                         "per_launch_flop": exec_flop},
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "clocks": clk,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+def _select(ab, p, Q, K, bufs):
+    import ctypes
+    lib = ab.lib()
+    st = ab._stream(Q.device)
+    ab._check(lib.ab_select(ctypes.byref(p.c()), ab._ptr(Q), ab._ptr(K), ab._ptr(bufs.P), None, None,
+                            ab._ptr(bufs.ws), bufs.ws.numel(), st), "ab_select")
+
+
+def _sample(ab, p, bufs):
+    import ctypes
+    lib = ab.lib()
+    st = ab._stream(bufs.P.device)
+    ab._check(lib.ab_sample(ctypes.byref(p.c()), ab._ptr(bufs.P), ab._ptr(bufs.idx), ab._ptr(bufs.pi_q32),
+                            ab._ptr(bufs.count), st), "ab_sample")
+
+
+def run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, steps):
+    import torch
+    Qh, Kh, Vh = (t.pin_memory() for t in (Qc, Kc, Vc))
+    Oh = torch.empty_like(Qc).pin_memory()
+    Qd, Kd, Vd = (torch.empty_like(Qc, device=dev) for _ in range(3))
+    stream = torch.cuda.current_stream(dev)
+    ab.ab_forward_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, bufs, dev)  # warm-up
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        ab.ab_forward_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, bufs, dev)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / steps
+    nbytes = Qc.numel() * 2
+    return {"value": round(dense_flop(w) / (ms * 1e-3) / 1e12, 3), "unit": UNIT,
+            "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": round(ms, 3),
+            "api": "ab_forward_host (pinned host Q/K/V in, host O out)"}
+
+
+def run_dense(ab, p, Q, K, V, dev, iters):
+    import torch
+    O = torch.empty_like(Q)
+    ab.ab_attention_dense(p, Q, K, V, out=O)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(iters):
+        ab.ab_attention_dense(p, Q, K, V, out=O)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    return t0.elapsed_time(t1) / iters
+
+
+# ---------------------------------------------------------- CPU oracle arm
+
+def cpu_sample_units(w, n_heads=4, n_blocks=16):
+    heads = sorted({int(round(k * (w.H - 1) / max(1, n_heads - 1))) for k in range(n_heads)})
+    blocks = sorted({int(round(k * (w.Nq - 1) / max(1, n_blocks - 1))) for k in range(n_blocks)})
+    return [(h, i) for h in heads for i in blocks]
+
+
+def cpu_baseline(w, args, Qc=None, Kc=None, Vc=None):
+    """The oracle, as it stands, on the host cores: IBCS + SIP + reweighted
+    attention for a bounded sample of (head, query block) units of the
+    workload, extrapolated to one layer."""
+    import oracle
+    from block_sparse_attention_queries_b200.synthetic import make_qkv
+    units = cpu_sample_units(w)
+    heads = sorted({h for h, _ in units})
+    # inputs of the sampled heads only (same generator, same seed)
+    if Qc is None:
+        from block_sparse_attention_queries_b200.synthetic import make_workload_qkv
+        Qc, Kc, Vc = make_workload_qkv(w)
+    Qn = {h: Qc[0, h].float().numpy() for h in heads}
+    Kn = {h: Kc[0, h].float().numpy() for h in heads}
+    Vn = {h: Vc[0, h].float().numpy() for h in heads}
+    Kb = oracle.budget(w.Nkv, w.keep_ratio)
+    threads = os.cpu_count() or 1
+
+    def one(u):
+        h, i = u
+        P = oracle.select_head(Qn[h], Kn[h], w.q_block, w.kv_block, w.C, w.kmeans_iters, rows=[i])
+        idx, pq, n = oracle.sip_row(P[0].astype(np.float32), Kb, 42, 0, h, i)
+        oracle.ht_attention_block(Qn[h], Kn[h], Vn[h], w.q_block, w.kv_block, i, idx, pq, n)
+        return n
+
+    t = time.perf_counter()
+    oracle.run_units(one, units, threads)
+    wall = time.perf_counter() - t
+    total_units = w.B * w.H * w.Nq
+    ms_layer = wall * 1e3 * total_units / len(units)
+    return {"value": round(dense_flop(w) / (ms_layer * 1e-3) / 1e12, 6), "unit": UNIT,
+            "cores": threads, "kind": "oracle",
+            "sample": f"{len(units)} (head, query block) units of {total_units} (heads {heads}), "
+                      f"select+sample+attention, {wall:.2f} s wall on {threads} threads; "
+                      f"ms/layer extrapolated = wall x {total_units}/{len(units)}",
+            "ms_per_layer_extrapolated": round(ms_layer, 1)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    from block_sparse_attention_queries_b200.synthetic import make_workload_qkv
+    w = workload()
+    Qc, Kc, Vc = make_workload_qkv(w)
+    vals = []
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(w, args, Qc, Kc, Vc)
+        vals.append(last["ms_per_layer_extrapolated"])
+    ms = statistics.mean(vals)
+    value = dense_flop(w) / (ms * 1e-3) / 1e12
+    return {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": config_dict(w, {"parallelism": "host threads"}),
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                             "sample": last["sample"]},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()
