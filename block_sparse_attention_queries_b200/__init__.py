@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "AB_OK", 1: "AB_ERR_INVALID_ARG", 2: "AB_ERR_UNSUPPORTED", 3:
 # every symbol include/ab.h declares
 EXPORTS = ("ab_budget", "ab_workspace_size", "ab_select", "ab_sample", "ab_attention",
            "ab_attention_dense", "ab_forward", "ab_forward_host", "ab_get_device_error",
-           "ab_status_string")
+           "ab_status_string", "ab_select_static")
 
 
 class AbError(RuntimeError):
@@ -100,11 +100,12 @@ def lib(path: str = LIB_PATH):
         L.ab_attention_dense.argtypes = [P, vp, vp, vp, vp, vp]
         L.ab_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ab_forward_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.ab_select_static.argtypes = [P, vp, vp, vp, vp, vp, vp]
         L.ab_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
         L.ab_status_string.argtypes = [ctypes.c_int]
         L.ab_status_string.restype = ctypes.c_char_p
         for name in ("ab_workspace_size", "ab_select", "ab_sample", "ab_attention", "ab_attention_dense",
-                     "ab_forward", "ab_forward_host", "ab_get_device_error"):
+                     "ab_forward", "ab_forward_host", "ab_get_device_error", "ab_select_static"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -159,6 +160,22 @@ def ab_select(p: Params, Q, K, workspace=None, want_centroids=False):
     ws = alloc_workspace(p, dev) if workspace is None else workspace
     _check(lib().ab_select(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(P), _ptr(cent), _ptr(cnt), _ptr(ws),
                            ws.numel(), _stream(dev)), "ab_select")
+    return (P, cent, cnt) if want_centroids else P
+
+
+def ab_select_static(p: Params, Q, K, want_centroids=False):
+    """ab_select with the library's own fixed device scratch: no workspace is
+    allocated (the outputs still are, here, by torch).  For callers that
+    cannot allocate device memory; see include/ab.h for the size limit and the
+    rule that overlapping calls race."""
+    import torch
+    _check_qkv(p, Q, K)
+    dev = Q.device
+    P = torch.empty(p.B, p.H, p.Nq, p.Nkv, dtype=torch.float32, device=dev)
+    cent = torch.empty(p.B, p.H, p.Nq, p.C, p.d, dtype=torch.float32, device=dev) if want_centroids else None
+    cnt = torch.empty(p.B, p.H, p.Nq, p.C, dtype=torch.int32, device=dev) if want_centroids else None
+    _check(lib().ab_select_static(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(P), _ptr(cent), _ptr(cnt),
+                                  _stream(dev)), "ab_select_static")
     return (P, cent, cnt) if want_centroids else P
 
 

@@ -247,6 +247,29 @@ ab_status do_attention(const Dims& d, const void* Q, const void* K, const void* 
                     : run_attention<64>(d, Q, K, V, idx, pi_q32, count, O, dense, st);
 }
 
+// ------------------------------------------- scratch for ab_select_static
+// One file-scope device array serves every ab_select_static call on a device.
+// Host code cannot use the symbol itself as a device address; its address is
+// looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_select_scratch[AB_SELECT_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_select_scratch on the current device (nullptr on failure).
+void* static_scratch_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess || !ptr) return nullptr;
+    g_scratch_addr[dev] = ptr;
+  }
+  return g_scratch_addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -329,6 +352,18 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
   if (s != AB_OK) return s;
   if (cudaMemcpyAsync(O_host, O, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return AB_ERR_CUDA;
   return AB_OK;
+}
+
+ab_status ab_select_static(const ab_params* p, const void* Q, const void* K, float* P, float* centroids,
+                           int32_t* counts, void* stream) {
+  Dims d;
+  const ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  if (workspace_layout(d).total > size_t(AB_SELECT_STATIC_SCRATCH_BYTES)) return AB_ERR_WORKSPACE;
+  void* scratch = static_scratch_current_device();
+  if (!scratch) return AB_ERR_CUDA;
+  return do_select(d, Q, K, P, centroids, counts, scratch, size_t(AB_SELECT_STATIC_SCRATCH_BYTES),
+                   static_cast<cudaStream_t>(stream));
 }
 
 ab_status ab_get_device_error(void* stream, int32_t* code) {

@@ -37,7 +37,8 @@
  *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  *    Every call only enqueues work on it and returns; results are ready when
  *    the stream reaches them.  The library keeps no state between calls other
- *    than the device error word.
+ *    than the device error word and the fixed scratch array behind
+ *    ab_select_static.
  *  - Errors: arguments are checked on the host before anything is launched;
  *    a bad argument returns AB_ERR_INVALID_ARG (or AB_ERR_UNSUPPORTED for a
  *    valid but unimplemented size) and enqueues nothing.  AB_ERR_CUDA reports
@@ -185,6 +186,38 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
                           void* O_host, void* Q, void* K, void* V, float* P, int32_t* idx,
                           uint32_t* pi_q32, int32_t* count, void* O, void* workspace, size_t ws_bytes,
                           void* stream);
+
+/*
+ * Size of the device array behind ab_select_static, in bytes (48 MiB).
+ */
+#define AB_SELECT_STATIC_SCRATCH_BYTES (48u * 1024u * 1024u)
+
+/*
+ * ab_select without a caller-supplied workspace, for callers that cannot
+ * allocate device memory: code running inside a host framework that owns
+ * every device allocation (a plugin under an inference engine's memory
+ * planner), or code that must not block, since cudaMalloc and cudaFree can
+ * synchronise the device.  The paper has no counterpart: this is an
+ * interface choice of this library, not part of the method.
+ *
+ * Same arguments, outputs and results as ab_select, minus the workspace.  The
+ * scratch is one array of AB_SELECT_STATIC_SCRATCH_BYTES in device memory,
+ * defined at file scope in the library, so every GPU that loads the library
+ * holds it until the process exits.  A problem whose ab_workspace_size
+ * exceeds that limit is rejected with AB_ERR_WORKSPACE before anything is
+ * enqueued (the Wan2.1-480p layer, 42 MB, fits; the HunyuanVideo-720p layer,
+ * 91 MB, does not).  Nothing is allocated or freed, by this call or by the
+ * library on its behalf.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call on a device shares the one array and leaves its contents behind;
+ * nothing in it needs to start at zero, because each call writes every byte
+ * it reads.  Calls whose work overlaps on the GPU (other streams, other host
+ * threads) race on the array: order them on one stream or synchronise.
+ */
+ab_status ab_select_static(const ab_params* p, const void* Q, const void* K, float* P, float* centroids,
+                           int32_t* counts, void* stream);
 
 /*
  * Reads and clears the device error word of the current device, after
