@@ -35,9 +35,10 @@ UNIT = "TFLOP/s"
 WORKLOAD = "wan2.1-14b-480p-self-attention"
 
 
-def workload():
+def workload(heads=None):
     from block_sparse_attention_queries_b200.synthetic import WORKLOADS
-    return WORKLOADS["wan480"]
+    w = WORKLOADS["wan480"]
+    return w if not heads else w.with_(H=heads)
 
 
 def dense_flop(w) -> float:
@@ -147,7 +148,7 @@ def run_ours(args):
         dist.init_process_group("nccl", rank=rank, world_size=world, device_id=dev,
                                 timeout=datetime.timedelta(seconds=120))
 
-    w = workload()
+    w = workload(args.heads)
     p = ab.Params.of(w, seed=42)
     # weak scaling: every rank runs its own layer (independent batch element)
     Qc, Kc, Vc = make_workload_qkv(w, seed=1234 + rank)
@@ -234,10 +235,13 @@ def run_ours(args):
 
     out = None
     if rank == 0:
-        # e2e through the public C ABI with host buffers (copies inside the region)
-        e2e = run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, max(2, min(args.steps, 5)))
-        dense_ms = run_dense(ab, p, Q, K, V, dev, 3)
-        cpu = cpu_baseline(w, args)
+        if args.no_extras:
+            e2e, dense_ms, cpu = None, float("nan"), None
+        else:
+            # e2e through the public C ABI with host buffers (copies inside the region)
+            e2e = run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, max(2, min(args.steps, 5)))
+            dense_ms = run_dense(ab, p, Q, K, V, dev, 3)
+            cpu = cpu_baseline(w, args, Qc, Kc, Vc)
         out = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
@@ -368,7 +372,7 @@ def run_reference(args):
     if rank != 0:
         return None
     from block_sparse_attention_queries_b200.synthetic import make_workload_qkv
-    w = workload()
+    w = workload(args.heads)
     Qc, Kc, Vc = make_workload_qkv(w)
     vals = []
     last = None
@@ -393,6 +397,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run a smaller case of the same layer with this many heads (profiling only)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the end-to-end, dense and CPU-baseline legs (profiling only)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
