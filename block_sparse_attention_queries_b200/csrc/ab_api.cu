@@ -109,6 +109,22 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   return r == CUDA_SUCCESS;
 }
 
+// K or V ([B*H, L, d] bf16, L % 8 == 0) viewed as {64, 8 rows, d/64 halves,
+// L/8 row groups, B*H}: one box of {64, 8, d/64, box_groups, 1} holds
+// 8*box_groups whole rows, laid out [group][half][row][128 B].
+bool make_map_grouped(CUtensorMap* m, const void* base, uint64_t d, uint64_t L, uint64_t BH, uint32_t box_groups) {
+  auto fn = encode_fn();
+  if (!fn || L % 8 != 0) return false;
+  const cuuint64_t dims[5] = {64, 8, d / 64, L / 8, BH};
+  const cuuint64_t strides[4] = {d * 2, 128, 8 * d * 2, L * d * 2};
+  const cuuint32_t box[5] = {64, 8, uint32_t(d / 64), box_groups, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -190,10 +206,16 @@ template <int D>
 ab_status run_attention(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* idx,
                         const uint32_t* pi_q32, const int32_t* count, void* O, bool dense, cudaStream_t st) {
   const int kvb = dense ? 128 : d.kv_block;
+  const bool grouped = (d.L % 8) == 0;
   CUtensorMap tmQ, tmK, tmV;
   if (!make_map(&tmQ, Q, D, d.L, d.BH, 128)) return AB_ERR_CUDA;
-  if (!make_map(&tmK, K, D, d.L, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
-  if (!make_map(&tmV, V, D, d.L, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
+  if (grouped) {
+    if (!make_map_grouped(&tmK, K, D, d.L, d.BH, uint32_t(kvb / 8))) return AB_ERR_CUDA;
+    if (!make_map_grouped(&tmV, V, D, d.L, d.BH, uint32_t(kvb / 8))) return AB_ERR_CUDA;
+  } else {
+    if (!make_map(&tmK, K, D, d.L, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
+    if (!make_map(&tmV, V, D, d.L, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
+  }
   AttnArgs a{};
   a.BH = d.BH; a.H = d.H; a.L = d.L; a.Nq = d.Nq; a.Nkv = dense ? (d.L + 127) / 128 : d.Nkv;
   a.q_block = d.q_block;
@@ -203,14 +225,23 @@ ab_status run_attention(const Dims& d, const void* Q, const void* K, const void*
   const int smem = AttnSmem<D>::kAlloc;
   auto launch = [&](auto kern) -> ab_status {
     if (set_smem(kern, smem) != cudaSuccess) return AB_ERR_CUDA;
-    kern<<<unsigned(d.BH * d.Nq), 192, smem, st>>>(tmQ, tmK, tmV, a);
+    // one CTA per pair of query blocks (2k, 2k+1) of a (b, h)
+    kern<<<unsigned(d.BH * ((d.Nq + 1) / 2)), 320, smem, st>>>(tmQ, tmK, tmV, a);
     return launch_status();
   };
+  if (grouped) {
+    switch (kvb) {
+      case 16: return launch(ab_attention_kernel<D, 16, true>);
+      case 32: return launch(ab_attention_kernel<D, 32, true>);
+      case 64: return launch(ab_attention_kernel<D, 64, true>);
+      default: return launch(ab_attention_kernel<D, 128, true>);
+    }
+  }
   switch (kvb) {
-    case 16: return launch(ab_attention_kernel<D, 16>);
-    case 32: return launch(ab_attention_kernel<D, 32>);
-    case 64: return launch(ab_attention_kernel<D, 64>);
-    default: return launch(ab_attention_kernel<D, 128>);
+    case 16: return launch(ab_attention_kernel<D, 16, false>);
+    case 32: return launch(ab_attention_kernel<D, 32, false>);
+    case 64: return launch(ab_attention_kernel<D, 64, false>);
+    default: return launch(ab_attention_kernel<D, 128, false>);
   }
 }
 

@@ -10,25 +10,34 @@
 // tiling mentioned on the Cross-Attention glossary page ("Sıkça Sorulan
 // Sorular").
 //
-// One CTA computes one query block of one (b, h): a 128-row query tile Q (rows
-// beyond the block are computed and discarded).  Its list of kept KV blocks is
-// consumed in tiles of 128 keys: 128 / kvb list entries per tile, each gathered
-// by TMA into consecutive rows of the K and V tiles.  Per tile:
-//   S = Q K^T            tcgen05, M=128 N=128 K=d, fp32 accumulator in TMEM
+// One CTA computes two query blocks ("streams" 0 and 1, query blocks 2k and
+// 2k+1 of one (b, h)), each a 128-row query tile (rows beyond the block are
+// computed and discarded).  A stream's list of kept KV blocks is consumed in
+// tiles of 128 keys: 128 / KVB list entries per tile, each gathered by TMA
+// into consecutive rows of the K and V tiles.  Per tile of stream s:
+//   S_s = Q_s K^T        tcgen05 (A, B in shared memory), M=128 N=128 K=d
 //   x = S log2(e)/sqrt(d) + log2(1/pi_slot)   (masked keys -> -inf)
-//   P = exp2(x - m)      bf16, written to shared memory (128B swizzle)
-//   O += P V             tcgen05, M=128 N=d K=128, fp32 accumulator in TMEM
+//   P_s = exp2(x - m)    bf16, stored back into TMEM over S_s
+//   O_s += P_s V         tcgen05 (A = P_s in TMEM, B = V in shared memory)
 // Weighting every term of block j by 1/pi_j is the additive bias log2(1/pi_j)
 // inside the exponent, so the weights enter the running max and sum for free.
-// The reference max m is only moved when a row max exceeds it by more than 8
-// (factor 256), so O is rescaled in TMEM only on those rare tiles; the final
-// O / l is unchanged by the choice of m.
+// The reference max m moves only when a row max passes it by more than 8
+// (factor 256); O_s is then rescaled in TMEM by the softmax warps themselves.
 //
-// Warp roles (192 threads): warps 0-3 softmax + epilogue (warp w owns TMEM
-// lanes 32w..32w+31, thread = query row), warp 4 TMA producer, warp 5 MMA
-// issuer and TMEM owner.  K tiles use a 3-deep ring (released when S is done),
-// V tiles a 2-deep ring (released when P V is done), S is double-buffered in
-// TMEM so that S(t+1) is computed while the softmax of tile t runs.
+// The two streams ping-pong: while the softmax warps of one stream work, the
+// tensor core runs the other stream's MMAs.  The MMA warp issues, per tile of
+// stream s, O_s += P_s V and then S_s(t+1) = Q_s K(t+1)^T into the same TMEM
+// columns; MMAs issued by one thread execute in order, so the next S never
+// overwrites P before the P V product has read it, and a commit after S_s(t+1)
+// also guarantees that O_s(t) is complete when the softmax reads S_s(t+1).
+//
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d),
+// O_1 [256+d, 256+2d); P_s occupies the first 64 columns of S_s.
+// Warps (320 threads): 0-3 softmax + epilogue of stream 0, 4-7 of stream 1
+// (warp w owns TMEM lanes 32(w%4)..+31, thread = query row), 8 TMA producer,
+// 9 MMA issuer and TMEM owner.  Tiles of the two streams are interleaved in
+// one order ("merged order": 0,1,0,1,... then the longer stream alone) that
+// the producer, the MMA warp and the K / V rings share.
 #pragma once
 
 #include "ab_ptx.cuh"
@@ -37,7 +46,7 @@ namespace ab {
 
 struct AttnArgs {
   int BH, H, L, Nq, Nkv;
-  int q_block;   // 64 or 128
+  int q_block;  // 64 or 128
   const int32_t* idx;
   const uint32_t* pi_q32;
   const int32_t* count;
@@ -48,19 +57,17 @@ struct AttnArgs {
 template <int D>
 struct AttnSmem {
   static constexpr int kSlabs = D / 64;
-  static constexpr int kSlab = 128 * 128;            // one 128-row x 128-byte slab
-  static constexpr int kTile = kSlabs * kSlab;       // 128 rows x D bf16
+  static constexpr int kSlab = 128 * 128;       // one 128-row x 128-byte slab
+  static constexpr int kTile = kSlabs * kSlab;  // 128 rows x D bf16
   static constexpr int kKStages = 3;
   static constexpr int kVStages = 2;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTile;
+  static constexpr int kOffQ = 0;  // two Q tiles
+  static constexpr int kOffK = kOffQ + 2 * kTile;
   static constexpr int kOffV = kOffK + kKStages * kTile;
-  static constexpr int kOffP = kOffV + kVStages * kTile;
-  static constexpr int kOffMeta = kOffP + 2 * kSlab;  // P: 128 x 128 bf16
-  // per V stage: 8 slot biases (log2 1/pi) and 8 valid-key counts
-  static constexpr int kMetaBytes = kVStages * 64;
-  static constexpr int kOffBar = kOffMeta + kMetaBytes;
-  static constexpr int kNumBars = 16;
+  static constexpr int kOffMeta = kOffV + kVStages * kTile;  // per K stage: 8 biases, 8 valid counts
+  static constexpr int kMetaStride = 64;
+  static constexpr int kOffBar = kOffMeta + kKStages * kMetaStride;
+  static constexpr int kNumBars = 20;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
@@ -68,15 +75,15 @@ struct AttnSmem {
 
 // barrier indices
 enum : int {
-  kBarQ = 0,
-  kBarKFull = 1,   // 3
-  kBarKEmpty = 4,  // 3
-  kBarVFull = 7,   // 2
-  kBarVEmpty = 9,  // 2
-  kBarSFull = 11,  // 2
-  kBarPFull = 13,
-  kBarODone = 14,
-  kBarDrain = 15,
+  kBarQ = 0,       // 2 (per stream)
+  kBarKFull = 2,   // 3
+  kBarKEmpty = 5,  // 3 (128 arrivals: the softmax warps of the tile's stream)
+  kBarVFull = 8,   // 2
+  kBarVEmpty = 10, // 2
+  kBarSFull = 12,  // 2 (per stream)
+  kBarPFull = 14,  // 2 (per stream, 128 arrivals)
+  kBarOFinal = 16, // 2 (per stream)
+  kBarDrain = 18,
 };
 
 // Warp-uniform bounded wait: every lane of the calling warp gets the same answer.
@@ -92,10 +99,33 @@ __device__ __forceinline__ bool lane0_wait(uint32_t bar, uint32_t parity, volati
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// Merged tile order of two streams with T0 and T1 tiles.
+struct Merge {
+  int T0, T1, m, longer;
+  __device__ Merge(int a, int b) : T0(a), T1(b), m(min(a, b)), longer(a >= b ? 0 : 1) {}
+  __device__ int total() const { return T0 + T1; }
+  __device__ void tile(int g, int& s, int& t) const {
+    if (g < 2 * m) {
+      s = g & 1;
+      t = g >> 1;
+    } else {
+      s = longer;
+      t = g - m;
+    }
+  }
+  __device__ int index(int s, int t) const { return t < m ? 2 * t + s : m + t; }
+};
+
 // D: head dim (64 or 128).  KVB: keys per list slot (16, 32, 64), or 128 for
 // dense attention (tile t = keys [128t, 128t+128), no list, no weights).
-template <int D, int KVB>
-__global__ void __launch_bounds__(192, 1)
+// kGrouped: K and V are read through a 5-D view {64 columns, 8 rows, d/64
+// halves, L/8 row groups, B*H} (needs L % 8 == 0), so that one TMA box
+// brings a whole KV block (both 64-column halves) into a K/V tile laid out as
+// [row group][half][8 rows][128 B]; otherwise one 3-D box per 64-column half,
+// into [half][128 rows][128 B].  Both are 128B-swizzled MMA operands; only the
+// strides in the descriptors differ.
+template <int D, int KVB, bool kGrouped>
+__global__ void __launch_bounds__(320, 1)
     ab_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using SM = AttnSmem<D>;
@@ -106,52 +136,59 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + SM::kOffBar;
   auto bar = [&](int k) { return bar0 + 8u * uint32_t(k); };
-  float* meta_bias = reinterpret_cast<float*>(smem + SM::kOffMeta);    // [2 stages] x 16, first 8 used
-  int* meta_valid = reinterpret_cast<int*>(smem + SM::kOffMeta + 32);  // same stride, offset by 8 words
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / a.Nq;
-  const int qi = blockIdx.x - bh * a.Nq;
+  const int pairs = (a.Nq + 1) / 2;
+  const int bh = blockIdx.x / pairs;
+  const int qi0 = (blockIdx.x - bh * pairs) * 2;
 
-  // list length and number of 128-key tiles of this query block
-  int cnt;
-  if (kDense) {
-    cnt = (a.L + 127) / 128;
-  } else {
-    cnt = a.count[blockIdx.x];
-    if (cnt < 0 || cnt > a.Nkv) {
-      if (threadIdx.x == 0) raise_error(AB_ERR_CAPACITY);
-      cnt = cnt < 0 ? 0 : a.Nkv;
+  // list length and number of 128-key tiles of each stream
+  int cnt[2], T[2];
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    const int qi = qi0 + s;
+    if (qi >= a.Nq) {
+      cnt[s] = 0;
+    } else if (kDense) {
+      cnt[s] = (a.L + 127) / 128;
+    } else {
+      int c = a.count[int64_t(bh) * a.Nq + qi];
+      if (c < 0 || c > a.Nkv) {
+        if (threadIdx.x == 0) raise_error(AB_ERR_CAPACITY);
+        c = c < 0 ? 0 : a.Nkv;
+      }
+      cnt[s] = c;
     }
+    T[s] = kDense ? cnt[s] : (cnt[s] + kSlots - 1) / kSlots;
   }
-  const int T = kDense ? cnt : (cnt + kSlots - 1) / kSlots;
-  const int64_t list_base = int64_t(blockIdx.x) * a.Nkv;
+  const Merge mg(T[0], T[1]);
+  const int G = mg.total();
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(kBarQ), 1);
-    for (int s = 0; s < 3; ++s) {
-      mbar_init(bar(kBarKFull + s), 1);
-      mbar_init(bar(kBarKEmpty + s), 1);
-    }
     for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarQ + s), 1);
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
       mbar_init(bar(kBarSFull + s), 1);
+      mbar_init(bar(kBarPFull + s), 128);
+      mbar_init(bar(kBarOFinal + s), 1);
     }
-    mbar_init(bar(kBarPFull), 128);
-    mbar_init(bar(kBarODone), 1);
+    for (int k = 0; k < 3; ++k) {
+      mbar_init(bar(kBarKFull + k), 1);
+      mbar_init(bar(kBarKEmpty + k), 128);
+    }
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
@@ -161,36 +198,44 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
-    // Lane s < kSlots owns list slot s of every tile: it reads the list entry,
-    // issues the TMA copies of that KV block's rows into the K (and one step
-    // later the V) tile, and hands the slot's weight and valid-key count to
-    // lane 0, which publishes them with the V tile.
+    // Lane e < kSlots owns list slot e of every tile: it reads the list entry
+    // and issues the TMA copies of that KV block's rows into rows
+    // [e*KVB, (e+1)*KVB) of the K tile, and one step later of the V tile.
+    // Lane 0 publishes the slots' weights and valid-key counts with the K tile.
     constexpr uint32_t kTileBytes = uint32_t(SM::kTile);
-    int issued_k[3] = {0, 0, 0}, issued_v[2] = {0, 0};
-    if (T > 0 && lane == 0) {
-      mbar_arrive_expect_tx(bar(kBarQ), kTileBytes);
-      for (int s = 0; s < SM::kSlabs; ++s)
-        tma_load_3d(sbase + SM::kOffQ + s * SM::kSlab, &tmQ, bar(kBarQ), s * 64, qi * a.q_block, bh);
+    int issued_k[3] = {0, 0, 0}, issued_v[2] = {0, 0}, issued_q[2] = {0, 0};
+    if (lane == 0) {
+      for (int s = 0; s < 2; ++s) {
+        if (T[s] == 0) continue;
+        mbar_arrive_expect_tx(bar(kBarQ + s), kTileBytes);
+        for (int sl = 0; sl < SM::kSlabs; ++sl)
+          tma_load_3d(sbase + SM::kOffQ + s * SM::kTile + sl * SM::kSlab, &tmQ, bar(kBarQ + s), sl * 64,
+                      (qi0 + s) * a.q_block, bh);
+        issued_q[s] = 1;
+      }
     }
-    int prev_row = 0, row = 0, prev_valid = 0, valid = 0;
-    float prev_bias = 0.f, bias = 0.f;
+    int prev_row = 0, row = 0;
     bool ok = true;
-    for (int u = 0; u <= T && ok; ++u) {
-      if (u < T) {
+    for (int u = 0; u <= G && ok; ++u) {
+      if (u < G) {
+        int s, t;
+        mg.tile(u, s, t);
+        float bias = 0.f;
+        int valid = 0;
         if (lane < kSlots) {
           if (kDense) {
-            row = u * 128;
+            row = t * 128;
             valid = min(128, a.L - row);
-            bias = 0.f;
           } else {
-            const int e = u * kSlots + lane;
+            const int e = t * kSlots + lane;
+            const int64_t base = (int64_t(bh) * a.Nq + qi0 + s) * a.Nkv;
             int j = -1;
             uint32_t pq = 0;
-            if (e < cnt) {
-              j = a.idx[list_base + e];
-              pq = a.pi_q32[list_base + e];
+            if (e < cnt[s]) {
+              j = a.idx[base + e];
+              pq = a.pi_q32[base + e];
               if (j < 0 || j >= a.Nkv) {
                 raise_error(AB_ERR_CAPACITY);
                 j = -1;
@@ -203,100 +248,127 @@ __global__ void __launch_bounds__(192, 1)
             } else {
               row = 0;  // empty slot: any in-range rows (finite data), fully masked
               valid = 0;
-              bias = 0.f;
             }
           }
         }
         const int ks = u % 3;
         if (!lane0_wait(bar(kBarKEmpty + ks), ((u / 3) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(bar(kBarKFull + ks), kTileBytes);
+        float b_all[kSlots];
+        int v_all[kSlots];
+#pragma unroll
+        for (int e = 0; e < kSlots; ++e) {
+          b_all[e] = __shfl_sync(0xffffffffu, bias, e);
+          v_all[e] = __shfl_sync(0xffffffffu, valid, e);
+        }
+        if (lane == 0) {
+          float* mb = reinterpret_cast<float*>(smem + SM::kOffMeta + ks * SM::kMetaStride);
+          int* mv = reinterpret_cast<int*>(smem + SM::kOffMeta + ks * SM::kMetaStride + 32);
+#pragma unroll
+          for (int e = 0; e < kSlots; ++e) {
+            mb[e] = b_all[e];
+            mv[e] = v_all[e];
+          }
+          mbar_arrive_expect_tx(bar(kBarKFull + ks), kTileBytes);
+        }
         __syncwarp();
         if (lane < kSlots) {
-          for (int s = 0; s < SM::kSlabs; ++s)
-            tma_load_3d(sbase + SM::kOffK + ks * SM::kTile + s * SM::kSlab + lane * KVB * 128, &tmK,
-                        bar(kBarKFull + ks), s * 64, row, bh);
+          if constexpr (kGrouped) {
+            tma_load_5d(sbase + SM::kOffK + ks * SM::kTile + lane * KVB * SM::kSlabs * 128, &tmK,
+                        bar(kBarKFull + ks), 0, 0, 0, row / 8, bh);
+          } else {
+            for (int sl = 0; sl < SM::kSlabs; ++sl)
+              tma_load_3d(sbase + SM::kOffK + ks * SM::kTile + sl * SM::kSlab + lane * KVB * 128, &tmK,
+                          bar(kBarKFull + ks), sl * 64, row, bh);
+          }
         }
         issued_k[ks] += 1;
       }
       if (u >= 1) {
-        const int t = u - 1;
-        const int vs = t & 1;
-        if (!lane0_wait(bar(kBarVEmpty + vs), ((t >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        float b_all[kSlots];
-        int v_all[kSlots];
-#pragma unroll
-        for (int s = 0; s < kSlots; ++s) {
-          b_all[s] = __shfl_sync(0xffffffffu, prev_bias, s);
-          v_all[s] = __shfl_sync(0xffffffffu, prev_valid, s);
-        }
-        if (lane == 0) {
-#pragma unroll
-          for (int s = 0; s < kSlots; ++s) {
-            meta_bias[vs * 16 + s] = b_all[s];
-            meta_valid[vs * 16 + s] = v_all[s];
-          }
-          mbar_arrive_expect_tx(bar(kBarVFull + vs), kTileBytes);
-        }
+        const int g = u - 1;
+        const int vs = g & 1;
+        if (!lane0_wait(bar(kBarVEmpty + vs), ((g >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(bar(kBarVFull + vs), kTileBytes);
         __syncwarp();
         if (lane < kSlots) {
-          for (int s = 0; s < SM::kSlabs; ++s)
-            tma_load_3d(sbase + SM::kOffV + vs * SM::kTile + s * SM::kSlab + lane * KVB * 128, &tmV,
-                        bar(kBarVFull + vs), s * 64, prev_row, bh);
+          if constexpr (kGrouped) {
+            tma_load_5d(sbase + SM::kOffV + vs * SM::kTile + lane * KVB * SM::kSlabs * 128, &tmV,
+                        bar(kBarVFull + vs), 0, 0, 0, prev_row / 8, bh);
+          } else {
+            for (int sl = 0; sl < SM::kSlabs; ++sl)
+              tma_load_3d(sbase + SM::kOffV + vs * SM::kTile + sl * SM::kSlab + lane * KVB * 128, &tmV,
+                          bar(kBarVFull + vs), sl * 64, prev_row, bh);
+          }
         }
         issued_v[vs] += 1;
       }
       prev_row = row;
-      prev_bias = bias;
-      prev_valid = valid;
     }
     if (!ok && lane == 0) {
       // let the copies already issued land before shared memory is released
-      for (int s = 0; s < 3; ++s)
-        if (issued_k[s]) mbar_wait_drain(bar(kBarKFull + s), (issued_k[s] - 1) & 1);
+      for (int k = 0; k < 3; ++k)
+        if (issued_k[k]) mbar_wait_drain(bar(kBarKFull + k), (issued_k[k] - 1) & 1);
+      for (int k = 0; k < 2; ++k)
+        if (issued_v[k]) mbar_wait_drain(bar(kBarVFull + k), (issued_v[k] - 1) & 1);
       for (int s = 0; s < 2; ++s)
-        if (issued_v[s]) mbar_wait_drain(bar(kBarVFull + s), (issued_v[s] - 1) & 1);
-      if (T > 0) mbar_wait_drain(bar(kBarQ), 0);
+        if (issued_q[s]) mbar_wait_drain(bar(kBarQ + s), 0);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA
-    if (T > 0 && lane == 0) {
+    if (G > 0 && lane == 0) {
       const uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);  // Q (K-major) x K tile (K-major)
-      const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // P (K-major) x V tile (MN-major)
-      const uint32_t tO = tmem + 256u;
-      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag);
-      auto issue_S = [&](int t) -> bool {
-        const int ks = t % 3;
-        if (!mbar_wait(bar(kBarKFull + ks), (t / 3) & 1, abort_flag)) return false;
+      const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // P (TMEM) x V tile (MN-major)
+      bool ok = true;
+      for (int s = 0; s < 2 && ok; ++s)
+        if (T[s] > 0) ok = mbar_wait(bar(kBarQ + s), 0, abort_flag);
+      auto issue_S = [&](int s, int t) -> bool {
+        const int g = mg.index(s, t);
+        const int ks = g % 3;
+        if (!mbar_wait(bar(kBarKFull + ks), (g / 3) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t qa = sbase + SM::kOffQ;
+        const uint32_t qa = sbase + SM::kOffQ + s * SM::kTile;
         const uint32_t kb = sbase + SM::kOffK + ks * SM::kTile;
+        // K tile: next 64 columns at kHalfK, 8-row groups kSboK apart
+        constexpr uint32_t kHalfK = kGrouped ? 1024u : uint32_t(SM::kSlab);
+        constexpr uint32_t kSboK = kGrouped ? uint32_t(SM::kSlabs) * 1024u : 1024u;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * SM::kSlab + (kk & 3) * 32;
-          mma_bf16_ss(tmem + uint32_t(t & 1) * 128u, smem_desc_sw128(qa + off, 16, 1024),
-                      smem_desc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          const uint32_t qoff = (kk >> 2) * SM::kSlab + (kk & 3) * 32;
+          const uint32_t koff = (kk >> 2) * kHalfK + (kk & 3) * 32;
+          mma_bf16_ss(tmem + uint32_t(s) * 128u, smem_desc_sw128(qa + qoff, 16, 1024),
+                      smem_desc_sw128(kb + koff, 16, kSboK), idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(kBarSFull + (t & 1)));
-        mma_commit(bar(kBarKEmpty + ks));
+        mma_commit(bar(kBarSFull + s));
         return true;
       };
-      if (ok) ok = issue_S(0);
-      if (ok && T > 1) ok = issue_S(1);
-      for (int t = 0; t < T && ok; ++t) {
-        if (!mbar_wait(bar(kBarPFull), t & 1, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(bar(kBarVFull + (t & 1)), (t >> 1) & 1, abort_flag)) { ok = false; break; }
+      // first tile of each stream, in merged order
+      for (int g = 0; g < min(G, 2) && ok; ++g) {
+        int s, t;
+        mg.tile(g, s, t);
+        if (t == 0) ok = issue_S(s, 0);
+      }
+      for (int g = 0; g < G && ok; ++g) {
+        int s, t;
+        mg.tile(g, s, t);
+        if (!mbar_wait(bar(kBarPFull + s), t & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(kBarVFull + (g & 1)), (g >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t pa = sbase + SM::kOffP;
-        const uint32_t vb = sbase + SM::kOffV + (t & 1) * SM::kTile;
+        const uint32_t vb = sbase + SM::kOffV + (g & 1) * SM::kTile;
+        const uint32_t tO = tmem + 256u + uint32_t(s * D);
+        const uint32_t tP = tmem + uint32_t(s) * 128u;
+        // V tile (MN-major): 16 keys per k-step, next 64 columns at kLboV, next 8 keys at kSboV
+        constexpr uint32_t kStepV = kGrouped ? 16u * uint32_t(SM::kSlabs) * 128u : 2048u;
+        constexpr uint32_t kLboV = kGrouped ? 1024u : uint32_t(SM::kSlab);
+        constexpr uint32_t kSboV = kGrouped ? uint32_t(SM::kSlabs) * 1024u : 1024u;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * SM::kSlab + (kk & 3) * 32;
-          mma_bf16_ss(tO, smem_desc_sw128(pa + aoff, 16, 1024), smem_desc_sw128(vb + kk * 2048, SM::kSlab, 1024),
-                      idO, (t > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tO, tP + uint32_t(kk * 8), smem_desc_sw128(vb + kk * kStepV, kLboV, kSboV), idO,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(kBarVEmpty + (g & 1)));
+        if (t + 1 < T[s]) {
+          ok = issue_S(s, t + 1);
+        } else {
+          mma_commit(bar(kBarOFinal + s));
         }
-        mma_commit(bar(kBarODone));
-        mma_commit(bar(kBarVEmpty + (t & 1)));
-        if (t + 2 < T) ok = issue_S(t + 2);
       }
       // every MMA issued above completes before TMEM and shared memory go away
       mma_commit(bar(kBarDrain));
@@ -304,43 +376,52 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------ softmax warps
-    const int r = threadIdx.x;  // query row within the tile == TMEM lane
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t tO = tmem + 256u + lane_base;
+    const int s = warp >> 2;       // stream
+    const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + uint32_t(s) * 128u + lane_base;
+    const uint32_t tO = tmem + 256u + uint32_t(s * D) + lane_base;
+    const int qi = qi0 + s;
     float m_use = -INFINITY;  // reference max (log2 domain)
     float l = 0.f;            // running sum of exp2(x - m_use)
     bool ok = true;
-    uint8_t* pbase = smem + SM::kOffP;
-    for (int t = 0; t < T && ok; ++t) {
-      const int sb = t & 1;
-      if (!warp_wait(bar(kBarSFull + sb), (t >> 1) & 1, abort_flag)) { ok = false; break; }
-      if (!warp_wait(bar(kBarVFull + sb), (t >> 1) & 1, abort_flag)) { ok = false; break; }
+    for (int t = 0; t < T[s] && ok; ++t) {
+      const int g = mg.index(s, t);
+      const int ks = g % 3;
+      if (!warp_wait(bar(kBarSFull + s), t & 1, abort_flag)) { ok = false; break; }
+      if (!warp_wait(bar(kBarKFull + ks), (g / 3) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float x[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + uint32_t(sb * 128 + c * 32) + lane_base, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(v[k]);
-      }
+      for (int c = 0; c < 4; ++c) tmem_ld32_nowait(tS + uint32_t(c * 32), reinterpret_cast<uint32_t*>(x) + c * 32);
+      // slot metadata of this tile (published with the K tile), then release the K stage
+      const float* mb = reinterpret_cast<const float*>(smem + SM::kOffMeta + ks * SM::kMetaStride);
+      const int* mv = reinterpret_cast<const int*>(smem + SM::kOffMeta + ks * SM::kMetaStride + 32);
       float s_bias[kSlots];
       int s_valid[kSlots];
+      bool full = true;
 #pragma unroll
-      for (int s = 0; s < kSlots; ++s) {
-        s_bias[s] = meta_bias[sb * 16 + s];
-        s_valid[s] = meta_valid[sb * 16 + s];
+      for (int e = 0; e < kSlots; ++e) {
+        s_bias[e] = mb[e];
+        s_valid[e] = mv[e];
+        full = full && (s_valid[e] == KVB);
       }
+      mbar_arrive(bar(kBarKEmpty + ks));
+      tmem_wait_ld();
       float rmax = -INFINITY;
+      if (full) {
 #pragma unroll
-      for (int k = 0; k < 128; ++k) {
-        constexpr int kb = KVB;
-        const int s = k / kb;
-        const int w = k % kb;
-        const float xv = (w < s_valid[s]) ? fmaf(x[k], a.scale_log2, s_bias[s]) : -INFINITY;
-        x[k] = xv;
-        rmax = fmaxf(rmax, xv);
+        for (int k = 0; k < 128; ++k) {
+          x[k] = fmaf(x[k], a.scale_log2, s_bias[k / KVB]);
+          rmax = fmaxf(rmax, x[k]);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 128; ++k) {
+          const int e = k / KVB, w = k % KVB;
+          x[k] = (w < s_valid[e]) ? fmaf(x[k], a.scale_log2, s_bias[e]) : -INFINITY;
+          rmax = fmaxf(rmax, x[k]);
+        }
       }
       // lazy reference max: move it only when the row max passes it by > 8
       const bool need = rmax > m_use + 8.f;
@@ -351,74 +432,69 @@ __global__ void __launch_bounds__(192, 1)
         l *= alpha;
       }
       const float mref = (m_use == -INFINITY) ? 0.f : m_use;
-      if (t > 0) {
-        // P V of the previous tile is done: P smem is free and O is stable
-        if (!warp_wait(bar(kBarODone), (t - 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tO + uint32_t(c * 32), v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
-            tmem_st32(tO + uint32_t(c * 32), v);
-          }
-          tmem_wait_st();
-        }
-      }
+      // P = exp2(x - m) as bf16 pairs over the first 64 columns of S_s
       float lsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint32_t pk[4];
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float p0 = ex2_approx(x[c * 8 + 2 * h] - mref);
-          const float p1 = ex2_approx(x[c * 8 + 2 * h + 1] - mref);
+        for (int k = 0; k < 32; ++k) {
+          const float p0 = ex2_approx(x[64 * h + 2 * k] - mref);
+          const float p1 = ex2_approx(x[64 * h + 2 * k + 1] - mref);
           lsum += p0 + p1;
-          pk[h] = pack_bf16x2(p0, p1);
+          pk[k] = pack_bf16x2(p0, p1);
         }
-        const uint32_t off = uint32_t(c >> 3) * SM::kSlab + sw128_offset(uint32_t(r), uint32_t(c & 7));
-        *reinterpret_cast<uint4*>(pbase + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        tmem_st32_ptr(tS + uint32_t(32 * h), pk);
       }
       l += lsum;
-      fence_proxy_async_smem();
+      // O_s is complete up to tile t-1 here (the commit behind S_s(t) covers it)
+      if (t > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + uint32_t(c * 32), o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(tO + uint32_t(c * 32), o);
+        }
+      }
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(kBarPFull));
+      mbar_arrive(bar(kBarPFull + s));
     }
     // ---------------------------------------------------------- epilogue
-    const int n_i = min(a.q_block, a.L - qi * a.q_block);
-    __nv_bfloat16* orow = a.O + (int64_t(bh) * a.L + int64_t(qi) * a.q_block + r) * D;
-    if (T > 0 && ok) ok = warp_wait(bar(kBarODone), (T - 1) & 1, abort_flag);
-    if (T > 0 && ok) {
-      tc_fence_after();
-      const float inv = 1.f / l;
+    if (qi < a.Nq) {
+      const int n_i = min(a.q_block, a.L - qi * a.q_block);
+      __nv_bfloat16* orow = a.O + (int64_t(bh) * a.L + int64_t(qi) * a.q_block + r) * D;
+      if (T[s] > 0 && ok) ok = warp_wait(bar(kBarOFinal + s), 0, abort_flag);
+      if (T[s] > 0 && ok) {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        uint32_t o[D];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tO + uint32_t(c * 32), v);
+        for (int c = 0; c < D / 32; ++c) tmem_ld32_nowait(tO + uint32_t(c * 32), o + c * 32);
         tmem_wait_ld();
         if (r < n_i) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
-            o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
-            o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
-            o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = o;
+          for (int q = 0; q < D / 8; ++q) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + q * 8) = w;
           }
         }
+      } else if (T[s] == 0 && r < n_i) {
+        for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4*>(orow + c * 8) = make_uint4(0, 0, 0, 0);
       }
-    } else if (T == 0 && r < n_i) {
-      for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4*>(orow + c * 8) = make_uint4(0, 0, 0, 0);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
