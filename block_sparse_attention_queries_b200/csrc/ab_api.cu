@@ -225,8 +225,13 @@ ab_status run_attention(const Dims& d, const void* Q, const void* K, const void*
   const int smem = AttnSmem<D>::kAlloc;
   auto launch = [&](auto kern) -> ab_status {
     if (set_smem(kern, smem) != cudaSuccess) return AB_ERR_CUDA;
+    // The kernel re-balances registers between its warpgroups; that only
+    // works if it is launched with the register count the split assumes.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return AB_ERR_CUDA;
+    if (fa.numRegs < kRegsLaunch) return AB_ERR_UNSUPPORTED;
     // one CTA per pair of query blocks (2k, 2k+1) of a (b, h)
-    kern<<<unsigned(d.BH * ((d.Nq + 1) / 2)), 320, smem, st>>>(tmQ, tmK, tmV, a);
+    kern<<<unsigned(d.BH * ((d.Nq + 1) / 2)), kAttnThreads, smem, st>>>(tmQ, tmK, tmV, a);
     return launch_status();
   };
   if (grouped) {

@@ -33,9 +33,11 @@
 //
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d),
 // O_1 [256+d, 256+2d); P_s occupies the first 64 columns of S_s.
-// Warps (320 threads): 0-3 softmax + epilogue of stream 0, 4-7 of stream 1
-// (warp w owns TMEM lanes 32(w%4)..+31, thread = query row), 8 TMA producer,
-// 9 MMA issuer and TMEM owner.  Tiles of the two streams are interleaved in
+// Warps (384 threads, three warpgroups): 0-3 softmax + epilogue of stream 0,
+// 4-7 of stream 1 (warp w owns TMEM lanes 32(w%4)..+31, thread = query row),
+// 8 TMA producer, 9 MMA issuer and TMEM owner, 10-11 idle.  The third
+// warpgroup hands registers to the two softmax warpgroups (setmaxnreg):
+// 384 x 168 at launch = 128 x kRegsCtl + 256 x kRegsSoftmax.  Tiles of the two streams are interleaved in
 // one order ("merged order": 0,1,0,1,... then the longer stream alone) that
 // the producer, the MMA warp and the K / V rings share.
 #pragma once
@@ -53,6 +55,13 @@ struct AttnArgs {
   __nv_bfloat16* O;
   float scale_log2;  // log2(e) / sqrt(d)
 };
+
+constexpr int kPolyEvery = 0;  // > 0: one column pair in kPolyEvery takes exp2 on the FMA pipe (off: measured slower)
+constexpr int kAttnThreads = 384;
+constexpr int kRegsLaunch = 168;   // registers per thread the kernel is launched with
+constexpr int kRegsCtl = 56;       // producer / MMA warpgroup after re-balancing
+constexpr int kRegsSoftmax = 224;  // softmax warpgroups after re-balancing
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kAttnThreads * kRegsLaunch, "register split exceeds the launch");
 
 template <int D>
 struct AttnSmem {
@@ -125,7 +134,7 @@ struct Merge {
 // into [half][128 rows][128 B].  Both are 128B-swizzled MMA operands; only the
 // strides in the descriptors differ.
 template <int D, int KVB, bool kGrouped>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     ab_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using SM = AttnSmem<D>;
@@ -197,7 +206,8 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) {
+    regs_dec<kRegsCtl>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     // Lane e < kSlots owns list slot e of every tile: it reads the list entry
@@ -317,6 +327,14 @@ __global__ void __launch_bounds__(320, 1)
     if (G > 0 && lane == 0) {
       const uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);  // Q (K-major) x K tile (K-major)
       const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // P (TMEM) x V tile (MN-major)
+      // descriptor bases, computed once; each MMA only adds its K offset
+      constexpr uint32_t kSboK = kGrouped ? uint32_t(SM::kSlabs) * 1024u : 1024u;
+      constexpr uint32_t kLboV = kGrouped ? 1024u : uint32_t(SM::kSlab);
+      constexpr uint32_t kSboV = kGrouped ? uint32_t(SM::kSlabs) * 1024u : 1024u;
+      const SmemDesc qdesc[2] = {smem_desc_base(sbase + SM::kOffQ, 16, 1024),
+                                 smem_desc_base(sbase + SM::kOffQ + SM::kTile, 16, 1024)};
+      const SmemDesc kdesc0 = smem_desc_base(sbase + SM::kOffK, 16, kSboK);
+      const SmemDesc vdesc0 = smem_desc_base(sbase + SM::kOffV, kLboV, kSboV);
       bool ok = true;
       for (int s = 0; s < 2 && ok; ++s)
         if (T[s] > 0) ok = mbar_wait(bar(kBarQ + s), 0, abort_flag);
@@ -325,17 +343,16 @@ __global__ void __launch_bounds__(320, 1)
         const int ks = g % 3;
         if (!mbar_wait(bar(kBarKFull + ks), (g / 3) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t qa = sbase + SM::kOffQ + s * SM::kTile;
-        const uint32_t kb = sbase + SM::kOffK + ks * SM::kTile;
         // K tile: next 64 columns at kHalfK, 8-row groups kSboK apart
         constexpr uint32_t kHalfK = kGrouped ? 1024u : uint32_t(SM::kSlab);
-        constexpr uint32_t kSboK = kGrouped ? uint32_t(SM::kSlabs) * 1024u : 1024u;
+        const SmemDesc qd = qdesc[s];
+        SmemDesc kd = kdesc0;
+        kd.lo += uint32_t(ks) * uint32_t(SM::kTile >> 4);
+        const uint32_t tSs = tmem + uint32_t(s) * 128u;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qoff = (kk >> 2) * SM::kSlab + (kk & 3) * 32;
-          const uint32_t koff = (kk >> 2) * kHalfK + (kk & 3) * 32;
-          mma_bf16_ss(tmem + uint32_t(s) * 128u, smem_desc_sw128(qa + qoff, 16, 1024),
-                      smem_desc_sw128(kb + koff, 16, kSboK), idS, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tSs, desc_at(qd, (kk >> 2) * SM::kSlab + (kk & 3) * 32),
+                      desc_at(kd, (kk >> 2) * kHalfK + (kk & 3) * 32), idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBarSFull + s));
         return true;
@@ -352,17 +369,15 @@ __global__ void __launch_bounds__(320, 1)
         if (!mbar_wait(bar(kBarPFull + s), t & 1, abort_flag)) { ok = false; break; }
         if (!mbar_wait(bar(kBarVFull + (g & 1)), (g >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t vb = sbase + SM::kOffV + (g & 1) * SM::kTile;
         const uint32_t tO = tmem + 256u + uint32_t(s * D);
         const uint32_t tP = tmem + uint32_t(s) * 128u;
         // V tile (MN-major): 16 keys per k-step, next 64 columns at kLboV, next 8 keys at kSboV
         constexpr uint32_t kStepV = kGrouped ? 16u * uint32_t(SM::kSlabs) * 128u : 2048u;
-        constexpr uint32_t kLboV = kGrouped ? 1024u : uint32_t(SM::kSlab);
-        constexpr uint32_t kSboV = kGrouped ? uint32_t(SM::kSlabs) * 1024u : 1024u;
+        SmemDesc vd = vdesc0;
+        vd.lo += uint32_t(g & 1) * uint32_t(SM::kTile >> 4);
+        mma_bf16_ts(tO, tP, desc_at(vd, 0), idO, t > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tO, tP + uint32_t(kk * 8), smem_desc_sw128(vb + kk * kStepV, kLboV, kSboV), idO,
-                      (t > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 1; kk < 8; ++kk) mma_bf16_ts(tO, tP + uint32_t(kk * 8), desc_at(vd, kk * kStepV), idO, 1u);
         mma_commit(bar(kBarVEmpty + (g & 1)));
         if (t + 1 < T[s]) {
           ok = issue_S(s, t + 1);
@@ -374,7 +389,9 @@ __global__ void __launch_bounds__(320, 1)
       mma_commit(bar(kBarDrain));
       mbar_wait_drain(bar(kBarDrain), 0);
     }
+  }
   } else {
+    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------ softmax warps
     const int s = warp >> 2;       // stream
     const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
@@ -408,43 +425,81 @@ __global__ void __launch_bounds__(320, 1)
       }
       mbar_arrive(bar(kBarKEmpty + ks));
       tmem_wait_ld();
-      float rmax = -INFINITY;
+      float lsum = 0.f;
+      bool need;
+      float alpha = 1.f;
       if (full) {
+        // Row max from per-slot maxima of the raw scores (scale > 0 commutes
+        // with max), then p = exp2(s * scale + (bias_slot - m)) with one packed
+        // FMA per pair of columns.
+        float rmax = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < 128; ++k) {
-          x[k] = fmaf(x[k], a.scale_log2, s_bias[k / KVB]);
-          rmax = fmaxf(rmax, x[k]);
+        for (int e = 0; e < kSlots; ++e) {
+          float mx = x[e * KVB];
+#pragma unroll
+          for (int k = 1; k + 1 < KVB; k += 2) mx = fmax3(mx, x[e * KVB + k], x[e * KVB + k + 1]);
+          mx = fmaxf(mx, x[e * KVB + KVB - 1]);
+          rmax = fmaxf(rmax, fmaf(mx, a.scale_log2, s_bias[e]));
         }
+        need = rmax > m_use + 8.f;
+        if (need) {
+          alpha = ex2_approx(m_use - rmax);  // 0 on the first tile
+          m_use = rmax;
+          l *= alpha;
+        }
+        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+        uint64_t acc2 = f2_pack(0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int c = 64 * h + 2 * k;
+            const float off = s_bias[c / KVB] - m_use;
+            float p0, p1;
+            f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), sc2, f2_pack(off, off)), p0, p1);
+            if (kPolyEvery > 0 && k % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+              exp2_poly2(p0, p1);  // a share of the exponentials on the FMA pipe
+            } else {
+              p0 = ex2_approx(p0);
+              p1 = ex2_approx(p1);
+            }
+            acc2 = f2_add(acc2, f2_pack(p0, p1));
+            pk[k] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32_ptr(tS + uint32_t(32 * h), pk);
+        }
+        float s0, s1;
+        f2_unpack(acc2, s0, s1);
+        lsum = s0 + s1;
       } else {
+        float rmax = -INFINITY;
 #pragma unroll
         for (int k = 0; k < 128; ++k) {
           const int e = k / KVB, w = k % KVB;
           x[k] = (w < s_valid[e]) ? fmaf(x[k], a.scale_log2, s_bias[e]) : -INFINITY;
           rmax = fmaxf(rmax, x[k]);
         }
-      }
-      // lazy reference max: move it only when the row max passes it by > 8
-      const bool need = rmax > m_use + 8.f;
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2_approx(m_use - rmax);  // 0 on the first tile
-        m_use = rmax;
-        l *= alpha;
-      }
-      const float mref = (m_use == -INFINITY) ? 0.f : m_use;
-      // P = exp2(x - m) as bf16 pairs over the first 64 columns of S_s
-      float lsum = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float p0 = ex2_approx(x[64 * h + 2 * k] - mref);
-          const float p1 = ex2_approx(x[64 * h + 2 * k + 1] - mref);
-          lsum += p0 + p1;
-          pk[k] = pack_bf16x2(p0, p1);
+        // lazy reference max: move it only when the row max passes it by > 8
+        need = rmax > m_use + 8.f;
+        if (need) {
+          alpha = ex2_approx(m_use - rmax);  // 0 on the first tile
+          m_use = rmax;
+          l *= alpha;
         }
-        tmem_st32_ptr(tS + uint32_t(32 * h), pk);
+        const float mref = (m_use == -INFINITY) ? 0.f : m_use;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float p0 = ex2_approx(x[64 * h + 2 * k] - mref);
+            const float p1 = ex2_approx(x[64 * h + 2 * k + 1] - mref);
+            lsum += p0 + p1;
+            pk[k] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32_ptr(tS + uint32_t(32 * h), pk);
+        }
       }
       l += lsum;
       // O_s is complete up to tile t-1 here (the commit behind S_s(t) covers it)
