@@ -29,6 +29,8 @@ from block_sparse_attention_queries_b200.synthetic import WORKLOADS, make_qkv, m
 def dev():
     if not torch.cuda.is_available():
         pytest.fail("no CUDA device")
+    from block_sparse_attention_queries_b200 import build as abbuild
+    abbuild.build()  # rebuilds only if a source is newer than libab.so
     ab.lib()  # the native library must load; there is no fallback
     return torch.device("cuda:0")
 
