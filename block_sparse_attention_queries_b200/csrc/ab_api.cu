@@ -189,7 +189,7 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, floa
     const int smem = ScSmem<D>::kAlloc;
     auto launch = [&](auto kern) -> ab_status {
       if (set_smem(kern, smem) != cudaSuccess) return AB_ERR_CUDA;
-      kern<<<grid, 160, smem, st>>>(tmCent, tmKsum, a);
+      kern<<<grid, 288, smem, st>>>(tmCent, tmKsum, a);
       return launch_status();
     };
     switch (d.C) {
@@ -267,7 +267,10 @@ ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q3
   a.P = P; a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
   a.H = d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
   a.seed_lo = uint32_t(d.seed); a.seed_hi = uint32_t(d.seed >> 32);
-  sip_kernel<<<unsigned(d.BH * d.Nq), 256, 0, st>>>(a);
+  const int smem = d.Nkv <= kSipSmemCap ? d.Nkv * 4 : 0;
+  if (smem > 48 * 1024 && cudaFuncSetAttribute(sip_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return AB_ERR_CUDA;
+  sip_kernel<<<unsigned(d.BH * d.Nq), 256, smem, st>>>(a);
   return launch_status();
 }
 

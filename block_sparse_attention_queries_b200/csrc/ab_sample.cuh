@@ -18,7 +18,9 @@
 //   this is tested without dividing: u < max(1, floor(X/S)) with X = R W 2^32
 //   holds iff u == 0 or (u + 1) S <= X.
 // Kept blocks are compacted in ascending j with a block-wide scan; each thread
-// owns 4 consecutive j per 1024-wide chunk (one Philox call per thread).
+// owns 4 consecutive j per 1024-wide chunk (one Philox call per thread).  The
+// quantised row W is read from global memory once and kept in shared memory
+// (rows up to kSipSmemCap entries; longer rows re-read P instead).
 #pragma once
 
 #include "ab_ptx.cuh"
@@ -80,9 +82,12 @@ __device__ __forceinline__ void block_sum2(uint64_t& a, uint64_t& b, uint64_t* r
   }
 }
 
+constexpr int kSipSmemCap = 16384;  // entries of W cached in shared memory (64 KB)
+
 __global__ void __launch_bounds__(256) sip_kernel(const SipArgs a) {
   __shared__ uint64_t red[16];
   __shared__ int scan[8];
+  extern __shared__ uint32_t wcache[];  // [Nkv] when Nkv <= kSipSmemCap
   const int row = blockIdx.x;
   const int b = row / (a.H * a.Nq);
   const int h = (row / a.Nq) % a.H;
@@ -90,6 +95,12 @@ __global__ void __launch_bounds__(256) sip_kernel(const SipArgs a) {
   const float* P = a.P + int64_t(row) * a.Nkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Nkv = a.Nkv;
+  const bool cached = Nkv <= kSipSmemCap;
+  if (cached) {
+    for (int j = tid; j < Nkv; j += 256) wcache[j] = uint32_t(quantise_w(__ldg(P + j)));
+    __syncthreads();
+  }
+  auto W = [&](int j) -> uint64_t { return cached ? uint64_t(wcache[j]) : quantise_w(__ldg(P + j)); };
 
   // ---- capping threshold (fixed point; at most Nkv + 1 rounds)
   uint64_t theta = ~0ull;  // nothing capped
@@ -97,7 +108,7 @@ __global__ void __launch_bounds__(256) sip_kernel(const SipArgs a) {
   for (int round = 0; round <= Nkv + 1; ++round) {
     uint64_t ncap = 0, sum = 0;
     for (int j = tid; j < Nkv; j += 256) {
-      const uint64_t w = quantise_w(__ldg(P + j));
+      const uint64_t w = W(j);
       if (w >= theta) ncap += 1;
       else sum += w;
     }
@@ -126,7 +137,7 @@ __global__ void __launch_bounds__(256) sip_kernel(const SipArgs a) {
       for (int q = 0; q < 4; ++q) {
         const int j = j0 + q;
         if (j >= Nkv) break;
-        const uint64_t w = quantise_w(__ldg(P + j));
+        const uint64_t w = W(j);
         bool keep;
         uint32_t pq;
         if (w >= theta) {

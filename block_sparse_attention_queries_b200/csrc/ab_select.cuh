@@ -12,8 +12,8 @@
 //                 |mu_c|^2 - 2 q.mu_c with q.mu_c on the tensor cores (the
 //                 fp32 centroid split into bf16 hi + lo parts, two
 //                 accumulating MMAs, so the dot products keep ~16 bits);
-//                 argmin per query, then a deterministic ordered
-//                 per-cluster sum (ballot-ranked, ascending query order).
+//                 argmin per query, then the per-cluster sums as a second
+//                 product Q^T x onehot(assignment) with fp32 accumulation.
 //  score_kernel   S = mu kbar^T / sqrt(d) on the tensor cores for 128/C query
 //                 blocks at once (M = 128 centroid rows, N = 256 KV blocks per
 //                 chunk), per-centroid softmax over j in two passes (max and
@@ -74,23 +74,22 @@ __global__ void __launch_bounds__(256) ksum_kernel(const __nv_bfloat16* __restri
 template <int D>
 struct KmSmem {
   static constexpr int kSlabs = D / 64;
-  static constexpr int kOffQ = 0;                        // 128 x D bf16, SW128 slabs of 16 KB
-  static constexpr int kOffBhi = kOffQ + kSlabs * 16384; // 16 x D bf16, SW128 slabs of 2 KB
-  static constexpr int kOffBlo = kOffBhi + kSlabs * 2048;
-  static constexpr int kOffMu = kOffBlo + kSlabs * 2048; // fp32 [16][D]
-  static constexpr int kOffMusq = kOffMu + 16 * D * 4;   // fp32 [16]
-  static constexpr int kOffAssign = kOffMusq + 64;       // int [128]
-  static constexpr int kOffOrder = kOffAssign + 512;     // int [128]
-  static constexpr int kOffWcnt = kOffOrder + 512;       // int [4 warps][16]
-  static constexpr int kOffStart = kOffWcnt + 256;       // int [4][16] per-warp offsets + [17] starts
-  static constexpr int kOffBar = kOffStart + 256 + 128;
+  static constexpr int kOffQ = 0;                         // 128 x D bf16, SW128 slabs of 16 KB
+  static constexpr int kOffBhi = kOffQ + 2 * 16384;       // 16 x D bf16, SW128 slabs of 2 KB
+  static constexpr int kOffBlo = kOffBhi + 2 * 2048;
+  static constexpr int kOffOneHot = kOffBlo + 2 * 2048;   // 16 clusters x 128 queries bf16, 2 slabs of 2 KB
+  static constexpr int kOffMu = kOffOneHot + 2 * 2048;    // fp32 [16][D]
+  static constexpr int kOffMusq = kOffMu + 16 * D * 4;    // fp32 [16]
+  static constexpr int kOffWcnt = kOffMusq + 64;          // int [4 warps][16]
+  static constexpr int kOffCnt = kOffWcnt + 256;          // int [16]
+  static constexpr int kOffBar = kOffCnt + 64;
   static constexpr int kOffMisc = kOffBar + 16;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-// Element (row, e) of a 128B-swizzled K-major bf16 tile with 16 KB (or
-// `slab`-byte) slabs of 64 columns.
+// Element (row, e) of a 128B-swizzled K-major bf16 tile with `slab_bytes`
+// slabs of 64 columns.
 __device__ __forceinline__ float sw_tile_get(const uint8_t* base, int slab_bytes, int row, int e) {
   const int slab = e >> 6, col = e & 63;
   const uint32_t off = uint32_t(slab * slab_bytes) + sw128_offset(uint32_t(row), uint32_t(col >> 3)) +
@@ -98,8 +97,15 @@ __device__ __forceinline__ float sw_tile_get(const uint8_t* base, int slab_bytes
   return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
 }
 
-// One CTA (128 threads) per query block.  Outputs: centroids (fp32, optional),
-// counts (optional), and for the scorer the bf16 centroids and int counts.
+// One CTA (128 threads) per query block.  Per Lloyd iteration, two small
+// tensor-core products:
+//   distances  q . mu_c = Q (128 x d) x [mu_hi; mu_lo]^T (d x 16), thread q
+//              reads its 16 columns and takes argmin |mu_c|^2 - 2 q . mu_c;
+//   sums       sum_{q in c} q = Q^T (d x 128) x onehot (128 x 16): Q is read
+//              as an MN-major operand (d contiguous), so thread e receives the
+//              sums of dimension e for every cluster in 16 TMEM columns.
+// Outputs: centroids (fp32, optional), counts (optional), and for the scorer
+// the bf16 centroids and int counts.
 template <int D, int C>
 __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUtensorMap tmQ, int L, int Nq,
                                                      int q_block, int iters, float* __restrict__ cent_out,
@@ -112,11 +118,8 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
   const uint32_t sbase = smem_u32(smem);
   float* mu = reinterpret_cast<float*>(smem + SM::kOffMu);
   float* musq = reinterpret_cast<float*>(smem + SM::kOffMusq);
-  int* assign = reinterpret_cast<int*>(smem + SM::kOffAssign);
-  int* order = reinterpret_cast<int*>(smem + SM::kOffOrder);
-  int* wcnt = reinterpret_cast<int*>(smem + SM::kOffWcnt);    // [4][16]
-  int* woff = reinterpret_cast<int*>(smem + SM::kOffStart);   // [4][16]
-  int* cstart = woff + 64;                                    // [17]
+  int* wcnt = reinterpret_cast<int*>(smem + SM::kOffWcnt);  // [4][16]
+  int* cnt = reinterpret_cast<int*>(smem + SM::kOffCnt);    // [16]
   const uint32_t bar_q = sbase + SM::kOffBar, bar_mma = sbase + SM::kOffBar + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kOffMisc + 4);
@@ -133,13 +136,17 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), 32);
+    tmem_alloc(smem_u32(tmem_slot), 64);  // columns 0-15 distances, 16-31 sums (x32 loads reach 47)
     tmem_relinquish();
   }
+  // one-hot rows >= C stay zero
+  for (int k = tid; k < 2 * 2048 / 16; k += 128)
+    reinterpret_cast<uint4*>(smem + SM::kOffOneHot)[k] = make_uint4(0, 0, 0, 0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t tlane = uint32_t(warp * 32) << 16;
 
   if (tid == 0) {
     mbar_arrive_expect_tx(bar_q, SM::kSlabs * 16384);
@@ -162,7 +169,9 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
   }
   __syncthreads();
 
-  const uint32_t idesc = idesc_bf16_f32(128, 16, 0, 0);
+  const uint32_t id_dist = idesc_bf16_f32(128, 16, 0, 0);  // Q (K-major) x mu parts (K-major)
+  const uint32_t id_sum = idesc_bf16_f32(128, 16, 1, 0);   // Q^T (MN-major) x onehot (K-major)
+  uint32_t phase = 0;
   for (int it = 0; it < iters && ok; ++it) {
     // centroid tiles (bf16 hi and lo parts, 16 rows, K-major SW128) and |mu|^2
     for (int k = tid; k < 16 * (D / 8); k += 128) {
@@ -198,19 +207,20 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
         const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
         const uint32_t boff = (kk >> 2) * 2048 + (kk & 3) * 32;
         mma_bf16_ss(tmem, smem_desc_sw128(sbase + SM::kOffQ + aoff, 16, 1024),
-                    smem_desc_sw128(sbase + SM::kOffBhi + boff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                    smem_desc_sw128(sbase + SM::kOffBhi + boff, 16, 1024), id_dist, kk > 0 ? 1u : 0u);
         mma_bf16_ss(tmem, smem_desc_sw128(sbase + SM::kOffQ + aoff, 16, 1024),
-                    smem_desc_sw128(sbase + SM::kOffBlo + boff, 16, 1024), idesc, 1u);
+                    smem_desc_sw128(sbase + SM::kOffBlo + boff, 16, 1024), id_dist, 1u);
       }
       mma_commit(bar_mma);
     }
-    ok = mbar_wait(bar_mma, it & 1, abort_flag);
+    ok = mbar_wait(bar_mma, phase & 1, abort_flag);
+    ++phase;
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
     // dot products of this thread's query with the 16 centroid rows
     uint32_t dv[32];
-    tmem_ld32(tmem + (uint32_t(warp * 32) << 16), dv);
+    tmem_ld32(tmem + tlane, dv);
     tmem_wait_ld();
     int best = C;  // C marks "no query" (rows beyond the block)
     if (tid < n_i) {
@@ -225,40 +235,49 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
         }
       }
     }
-    assign[tid] = best;
-    // ordered bucket of each query: warp ballots give the rank inside the warp
-    int my_rank = 0;
+    // cluster sizes (ballots) and this query's one-hot column
 #pragma unroll
     for (int c = 0; c < C; ++c) {
       const uint32_t bal = __ballot_sync(0xffffffffu, best == c);
-      if (best == c) my_rank = __popc(bal & ((1u << lane) - 1u));
       if (lane == 0) wcnt[warp * 16 + c] = __popc(bal);
     }
+    {
+      const int q = tid;
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        const uint32_t off = uint32_t((q >> 6) * 2048) + sw128_offset(uint32_t(c), uint32_t((q & 63) >> 3)) +
+                             uint32_t((q & 7) * 2);
+        *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffOneHot + off) =
+            __float2bfloat16_rn(best == c ? 1.f : 0.f);
+      }
+    }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid < C) cnt[tid] = wcnt[tid] + wcnt[16 + tid] + wcnt[32 + tid] + wcnt[48 + tid];
     if (tid == 0) {
-      int run = 0;
-      for (int c = 0; c < C; ++c) {
-        cstart[c] = run;
-        for (int w = 0; w < 4; ++w) {
-          woff[w * 16 + c] = run;
-          run += wcnt[w * 16 + c];
-        }
-      }
-      cstart[C] = run;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)  // K = 128 queries, 16 per step
+        mma_bf16_ss(tmem + 16u, smem_desc_sw128(sbase + SM::kOffQ + kk * 2048, 16384, 1024),
+                    smem_desc_sw128(sbase + SM::kOffOneHot + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), id_sum,
+                    kk > 0 ? 1u : 0u);
+      mma_commit(bar_mma);
     }
-    __syncthreads();
-    if (best < C) order[woff[warp * 16 + best] + my_rank] = tid;
-    __syncthreads();
-    // new centroid = mean of the members, summed in ascending query order
-    for (int e = tid; e < D; e += 128) {
-      for (int c = 0; c < C; ++c) {
-        const int b0 = cstart[c], b1 = cstart[c + 1];
-        if (b1 == b0) continue;  // empty cluster keeps its centroid
-        float s = 0.f;
-        for (int k = b0; k < b1; ++k) s += sw_tile_get(qtile, 16384, order[k], e);
-        mu[c * D + e] = s / float(b1 - b0);
-      }
+    ok = mbar_wait(bar_mma, phase & 1, abort_flag);
+    ++phase;
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    tc_fence_after();
+    // new centroid = sum of members / count (thread e holds dimension e); an
+    // empty cluster keeps its centroid
+    uint32_t sv[32];
+    tmem_ld32(tmem + tlane + 16u, sv);
+    tmem_wait_ld();
+    if (tid < D) {
+#pragma unroll
+      for (int c = 0; c < C; ++c)
+        if (cnt[c] > 0) mu[c * D + tid] = __uint_as_float(sv[c]) / float(cnt[c]);
     }
     __syncthreads();
   }
@@ -271,16 +290,15 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
       cent_ws[row0 * D + k] = __float2bfloat16_rn(v);
     }
     if (tid < C) {
-      const int n_c = cstart[tid + 1] - cstart[tid];
-      if (counts_out) counts_out[row0 + tid] = n_c;
-      counts_ws[row0 + tid] = n_c;
+      if (counts_out) counts_out[row0 + tid] = cnt[tid];
+      counts_ws[row0 + tid] = cnt[tid];
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 32);
+    tmem_dealloc(tmem, 64);
   }
 }
 
@@ -293,8 +311,9 @@ struct ScSmem {
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kA;           // 2 stages
   static constexpr int kOffW = kOffB + 2 * kB;       // float [128] row weights
-  static constexpr int kOffBar = kOffW + 512;        // a_full, b_full[2], b_empty[2], s_full[2], t_free[2]
-  static constexpr int kOffMisc = kOffBar + 10 * 8;
+  static constexpr int kOffX = kOffW + 512;          // float [2 halves][2][128] max/sum exchange
+  static constexpr int kOffBar = kOffX + 2048;       // a_full, b_full[2], b_empty[2], s_full[2], t_free[2], drain, xch
+  static constexpr int kOffMisc = kOffBar + 12 * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -327,8 +346,12 @@ __device__ __forceinline__ void group_reduce_scatter(float (&v)[32], int lane) {
   }
 }
 
+// Warps 0-7 read the scores (warp w: TMEM lanes 32 (w % 4).., columns
+// [128 (w / 4), +128) of every 256-column chunk), warp 8 loads and issues the
+// MMAs.  The two column halves of a row keep separate running max / sum in
+// the first pass and merge them before the second.
 template <int D, int C>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(288, 1)
     score_kernel(const __grid_constant__ CUtensorMap tmCent, const __grid_constant__ CUtensorMap tmKsum,
                  const ScoreArgs a) {
   using SM = ScSmem<D>;
@@ -338,7 +361,7 @@ __global__ void __launch_bounds__(160, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + SM::kOffBar;
   auto bar = [&](int k) { return bar0 + 8u * uint32_t(k); };
-  enum { kA = 0, kBFull = 1, kBEmpty = 3, kSFull = 5, kTFree = 7, kDrain = 9 };
+  enum { kA = 0, kBFull = 1, kBEmpty = 3, kSFull = 5, kTFree = 7, kDrain = 9, kXch = 10 };
   float* roww = reinterpret_cast<float*>(smem + SM::kOffW);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kOffMisc + 4);
@@ -355,9 +378,10 @@ __global__ void __launch_bounds__(160, 1)
       mbar_init(bar(kBFull + s), 1);
       mbar_init(bar(kBEmpty + s), 1);
       mbar_init(bar(kSFull + s), 1);
-      mbar_init(bar(kTFree + s), 128);
+      mbar_init(bar(kTFree + s), 8);  // one arrival per reader warp
     }
     mbar_init(bar(kDrain), 1);
+    mbar_init(bar(kXch), 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -371,7 +395,7 @@ __global__ void __launch_bounds__(160, 1)
     }
     roww[tid] = w;
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -381,7 +405,7 @@ __global__ void __launch_bounds__(160, 1)
   const uint32_t tmem = *tmem_slot;
   const int total = 2 * nchunks;  // pass 0: max and sum; pass 1: values
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       bool ok = true;
       mbar_arrive_expect_tx(bar(kA), SM::kA);
@@ -422,9 +446,11 @@ __global__ void __launch_bounds__(160, 1)
       mbar_wait_drain(bar(kDrain), 0);
     }
   } else {
-    const int r = tid;  // centroid row == TMEM lane
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const int r = tid & 127;   // centroid row == TMEM lane
+    const int ch = warp >> 2;  // column half of every chunk
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const float w = roww[r];
+    float* xm = reinterpret_cast<float*>(smem + SM::kOffX);  // [2][2][128]: max, sum per half
     float M = -INFINITY, Z = 0.f;
     bool ok = true;
     for (int g = 0; g < total && ok; ++g) {
@@ -434,13 +460,26 @@ __global__ void __launch_bounds__(160, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + st), (g >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
+      if (g == nchunks) {
+        // merge the two halves' running max and sum before the second pass
+        xm[(0 * 2 + ch) * 128 + r] = M;
+        xm[(1 * 2 + ch) * 128 + r] = Z;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kXch));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kXch), 0, abort_flag));
+        if (!ok) break;
+        const float M2 = xm[(0 * 2 + (ch ^ 1)) * 128 + r], Z2 = xm[(1 * 2 + (ch ^ 1)) * 128 + r];
+        const float Mx = fmaxf(M, M2);  // at least one half has a valid column
+        Z = (M == -INFINITY ? 0.f : Z * ex2_approx(M - Mx)) + (M2 == -INFINITY ? 0.f : Z2 * ex2_approx(M2 - Mx));
+        M = Mx;
+      }
       const float inv_z = pass2 ? w / Z : 0.f;
 #pragma unroll 1
-      for (int piece = 0; piece < 8; ++piece) {
+      for (int piece = 0; piece < 4; ++piece) {
         uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + uint32_t(st * 256 + piece * 32), raw);
+        tmem_ld32(tmem + lane_base + uint32_t(st * 256 + ch * 128 + piece * 32), raw);
         tmem_wait_ld();
-        const int j0 = chunk * 256 + piece * 32;
+        const int j0 = chunk * 256 + ch * 128 + piece * 32;
         float v[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
@@ -453,11 +492,13 @@ __global__ void __launch_bounds__(160, 1)
           float pm = M;
 #pragma unroll
           for (int k = 0; k < 32; ++k) pm = fmaxf(pm, v[k]);
-          float s = 0.f;
+          if (pm != -INFINITY) {  // a piece entirely past Nkv changes nothing
+            float s = 0.f;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) s += ex2_approx(v[k] - pm);
-          Z = Z * ex2_approx(M - pm) + s;  // M = -inf on the first piece: factor 0
-          M = pm;
+            for (int k = 0; k < 32; ++k) s += ex2_approx(v[k] - pm);
+            Z = (M == -INFINITY ? 0.f : Z * ex2_approx(M - pm)) + s;
+            M = pm;
+          }
         } else {
 #pragma unroll
           for (int k = 0; k < 32; ++k) v[k] = ex2_approx(v[k] - M) * inv_z;
@@ -476,12 +517,13 @@ __global__ void __launch_bounds__(160, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(kTFree + st));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kTFree + st));
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
