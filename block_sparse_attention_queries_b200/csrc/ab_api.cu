@@ -267,10 +267,15 @@ ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q3
   a.P = P; a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
   a.H = d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
   a.seed_lo = uint32_t(d.seed); a.seed_hi = uint32_t(d.seed >> 32);
-  const int smem = d.Nkv <= kSipSmemCap ? d.Nkv * 4 : 0;
-  if (smem > 48 * 1024 && cudaFuncSetAttribute(sip_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return AB_ERR_CUDA;
-  sip_kernel<<<unsigned(d.BH * d.Nq), 256, smem, st>>>(a);
+  if (d.Nkv <= kSipSmemCap) {
+    const int smem = 16 * ((d.Nkv + 3) / 4);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(sip_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return AB_ERR_CUDA;
+    sip_kernel<true><<<unsigned(d.BH * d.Nq), kSipThreads, smem, st>>>(a);
+  } else {
+    sip_kernel<false><<<unsigned(d.BH * d.Nq), kSipThreads, 0, st>>>(a);
+  }
   return launch_status();
 }
 

@@ -226,9 +226,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         issued_q[s] = 1;
       }
     }
+    // List entries are fetched two tiles ahead of their use, so that the
+    // latency of the global loads overlaps the waits and copies of the
+    // tiles before.
+    auto fetch = [&](int u, int& j, uint32_t& pq) {
+      j = -1;
+      pq = 0;
+      if (!kDense && u < G && lane < kSlots) {
+        int s, t;
+        mg.tile(u, s, t);
+        const int e = t * kSlots + lane;
+        if (e < cnt[s]) {
+          const int64_t at = (int64_t(bh) * a.Nq + qi0 + s) * a.Nkv + e;
+          j = __ldg(a.idx + at);
+          pq = __ldg(a.pi_q32 + at);
+          if (j < 0 || j >= a.Nkv) {
+            raise_error(AB_ERR_CAPACITY);
+            j = -1;
+          }
+        }
+      }
+    };
+    int j_cur, j_next, j_far;
+    uint32_t pq_cur, pq_next, pq_far;
+    fetch(0, j_cur, pq_cur);
+    fetch(1, j_next, pq_next);
     int prev_row = 0, row = 0;
     bool ok = true;
     for (int u = 0; u <= G && ok; ++u) {
+      fetch(u + 2, j_far, pq_far);
       if (u < G) {
         int s, t;
         mg.tile(u, s, t);
@@ -238,27 +264,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (kDense) {
             row = t * 128;
             valid = min(128, a.L - row);
+          } else if (j_cur >= 0) {
+            row = j_cur * KVB;
+            valid = min(KVB, a.L - row);
+            bias = pq_cur == 0u ? 0.f : 32.f - log2f(float(pq_cur));  // log2(1/pi), Pi = pq or 2^32
           } else {
-            const int e = t * kSlots + lane;
-            const int64_t base = (int64_t(bh) * a.Nq + qi0 + s) * a.Nkv;
-            int j = -1;
-            uint32_t pq = 0;
-            if (e < cnt[s]) {
-              j = a.idx[base + e];
-              pq = a.pi_q32[base + e];
-              if (j < 0 || j >= a.Nkv) {
-                raise_error(AB_ERR_CAPACITY);
-                j = -1;
-              }
-            }
-            if (j >= 0) {
-              row = j * KVB;
-              valid = min(KVB, a.L - row);
-              bias = pq == 0u ? 0.f : 32.f - log2f(float(pq));  // log2(1/pi), Pi = pq or 2^32
-            } else {
-              row = 0;  // empty slot: any in-range rows (finite data), fully masked
-              valid = 0;
-            }
+            row = 0;  // empty slot: any in-range rows (finite data), fully masked
+            valid = 0;
           }
         }
         const int ks = u % 3;
@@ -312,6 +324,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         issued_v[vs] += 1;
       }
       prev_row = row;
+      j_cur = j_next;
+      pq_cur = pq_next;
+      j_next = j_far;
+      pq_next = pq_far;
     }
     if (!ok && lane == 0) {
       // let the copies already issued land before shared memory is released

@@ -17,10 +17,12 @@
 //   Philox4x32-10((j div 4, i, h, b), (seed lo, seed hi)).  For a free block
 //   this is tested without dividing: u < max(1, floor(X/S)) with X = R W 2^32
 //   holds iff u == 0 or (u + 1) S <= X.
-// Kept blocks are compacted in ascending j with a block-wide scan; each thread
-// owns 4 consecutive j per 1024-wide chunk (one Philox call per thread).  The
-// quantised row W is read from global memory once and kept in shared memory
-// (rows up to kSipSmemCap entries; longer rows re-read P instead).
+// Each thread owns 4 consecutive j per 1024-wide chunk (one Philox call per
+// thread and chunk).  Phases: (1) the quantised row is cached in shared memory
+// (rows up to kSipSmemCap entries; longer rows re-read P); (2) capping rounds,
+// one barrier each; (3) draws, with the kept j compacted in ascending order
+// by a block-wide scan; (4) Pi of the kept entries, one output position per
+// thread, so the exact division runs without divergence.
 #pragma once
 
 #include "ab_ptx.cuh"
@@ -54,40 +56,32 @@ struct SipArgs {
   uint32_t seed_lo, seed_hi;
 };
 
-__device__ __forceinline__ uint64_t quantise_w(float p) {
+__device__ __forceinline__ uint32_t quantise_w(float p) {
   const float s = floorf(p * 16777216.0f);
-  return s < 1.0f ? 1ull : uint64_t(s);
+  return s < 1.0f ? 1u : uint32_t(s);  // p <= 1, so s <= 2^24
 }
 
-// Block-wide sum of (count, sum) pairs over 256 threads.
-__device__ __forceinline__ void block_sum2(uint64_t& a, uint64_t& b, uint64_t* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    a += __shfl_xor_sync(0xffffffffu, a, o);
-    b += __shfl_xor_sync(0xffffffffu, b, o);
-  }
-  __syncthreads();
-  if (lane == 0) {
-    red[warp] = a;
-    red[8 + warp] = b;
-  }
-  __syncthreads();
-  a = 0;
-  b = 0;
-#pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    a += red[w];
-    b += red[8 + w];
-  }
+// a S <= X 2^32 for a < 2^32 + 1, S = S_hi 2^32 + S_lo < 2^64, X < 2^64:
+// a S = (a S_hi) 2^32 + a S_lo, compared without 128-bit products.
+// `a` is passed as a_minus_1 (so that a = 2^32 fits) .
+__device__ __forceinline__ bool mul_le_shift32(uint32_t a_minus_1, uint32_t S_hi, uint32_t S_lo, uint64_t X) {
+  const uint64_t t = uint64_t(a_minus_1) * S_lo + S_lo;  // a S_lo < 2^64
+  const uint64_t h = uint64_t(a_minus_1) * S_hi + S_hi;  // a S_hi
+  if (h > X) return false;
+  const uint64_t r = X - h;
+  return r >= (1ull << 32) || t <= (r << 32);
 }
 
+constexpr int kSipThreads = 256;
 constexpr int kSipSmemCap = 16384;  // entries of W cached in shared memory (64 KB)
 
-__global__ void __launch_bounds__(256) sip_kernel(const SipArgs a) {
-  __shared__ uint64_t red[16];
+template <bool kCached>
+__global__ void __launch_bounds__(kSipThreads) sip_kernel(const SipArgs a) {
+  __shared__ uint64_t red_sum[2][8];
+  __shared__ uint32_t red_cnt[2][8];
   __shared__ int scan[8];
-  extern __shared__ uint32_t wcache[];  // [Nkv] when Nkv <= kSipSmemCap
+  extern __shared__ uint4 wcache4[];  // [ceil(Nkv / 4)] when cached; entries >= Nkv hold 0
+  uint32_t* wcache = reinterpret_cast<uint32_t*>(wcache4);
   const int row = blockIdx.x;
   const int b = row / (a.H * a.Nq);
   const int h = (row / a.Nq) % a.H;
@@ -95,69 +89,98 @@ __global__ void __launch_bounds__(256) sip_kernel(const SipArgs a) {
   const float* P = a.P + int64_t(row) * a.Nkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Nkv = a.Nkv;
-  const bool cached = Nkv <= kSipSmemCap;
-  if (cached) {
-    for (int j = tid; j < Nkv; j += 256) wcache[j] = uint32_t(quantise_w(__ldg(P + j)));
+
+  // W of j0 .. j0 + 3 (j0 a multiple of 4, j0 < Nkv); entries >= Nkv read 0
+  auto load4 = [&](int j0, uint32_t (&w)[4]) {
+    if constexpr (kCached) {
+      const uint4 v = wcache4[j0 >> 2];
+      w[0] = v.x;
+      w[1] = v.y;
+      w[2] = v.z;
+      w[3] = v.w;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w[q] = j0 + q < Nkv ? quantise_w(__ldg(P + j0 + q)) : 0u;
+    }
+  };
+  if constexpr (kCached) {
+    const int n4 = (Nkv + 3) >> 2;
+    for (int k = tid; k < 4 * n4; k += kSipThreads) wcache[k] = k < Nkv ? quantise_w(__ldg(P + k)) : 0u;
     __syncthreads();
   }
-  auto W = [&](int j) -> uint64_t { return cached ? uint64_t(wcache[j]) : quantise_w(__ldg(P + j)); };
 
   // ---- capping threshold (fixed point; at most Nkv + 1 rounds)
-  uint64_t theta = ~0ull;  // nothing capped
+  uint32_t theta = 0xFFFFFFFFu;  // above every W: nothing capped
   uint64_t R = 0, S = 0;
   for (int round = 0; round <= Nkv + 1; ++round) {
-    uint64_t ncap = 0, sum = 0;
-    for (int j = tid; j < Nkv; j += 256) {
-      const uint64_t w = W(j);
-      if (w >= theta) ncap += 1;
-      else sum += w;
+    uint32_t ncap = 0;
+    uint64_t sum = 0;
+    for (int j0 = 4 * tid; j0 < Nkv; j0 += 4 * kSipThreads) {
+      uint32_t w[4];
+      load4(j0, w);
+      uint32_t part = 0;  // <= 4 * 2^24
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const bool cap = w[q] >= theta;
+        ncap += cap ? 1u : 0u;
+        part += cap ? 0u : w[q];
+      }
+      sum += part;
     }
-    block_sum2(ncap, sum, red);
-    R = uint64_t(a.Kb) - ncap;
-    S = sum;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ncap += __shfl_xor_sync(0xffffffffu, ncap, o);
+      sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    const int buf = round & 1;  // double buffer: one barrier per round
+    if (lane == 0) {
+      red_cnt[buf][warp] = ncap;
+      red_sum[buf][warp] = sum;
+    }
+    __syncthreads();
+    uint64_t nc = 0;
+    S = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      nc += red_cnt[buf][w];
+      S += red_sum[buf][w];
+    }
+    R = uint64_t(a.Kb) - nc;
     if (R == 0 || S == 0) break;
-    const uint64_t t_new = (S + R - 1) / R;  // R W >= S  <=>  W >= ceil(S / R)
+    // ceil(S / R): double quotient, then exact integer correction
+    uint64_t q = uint64_t(double(S) / double(R));
+    while (q * R > S) --q;
+    while ((q + 1) * R <= S) ++q;
+    const uint64_t t_new = q + (q * R != S ? 1u : 0u);  // R W >= S  <=>  W >= ceil(S / R)
     if (t_new >= theta) break;
-    theta = t_new;
+    theta = uint32_t(t_new);  // t_new < theta <= 2^32 - 1
   }
 
   // ---- draws and ordered compaction, 4 consecutive j per thread per chunk
   const uint32_t k0 = a.seed_lo, k1 = a.seed_hi;
+  const uint32_t S_hi = uint32_t(S >> 32), S_lo = uint32_t(S);
+  const uint32_t R32 = uint32_t(R);  // R <= Kb < 2^31
   int32_t* out_idx = a.idx + int64_t(row) * Nkv;
   uint32_t* out_pi = a.pi_q32 + int64_t(row) * Nkv;
   int base = 0;
-  for (int c0 = 0; c0 < Nkv; c0 += 1024) {
+  for (int c0 = 0; c0 < Nkv; c0 += 4 * kSipThreads) {
     const int j0 = c0 + 4 * tid;
     uint32_t keep_mask = 0;
-    uint32_t pis[4] = {0, 0, 0, 0};
     if (j0 < Nkv) {
       const uint4 u4 = philox4x32_10(make_uint4(uint32_t(j0 >> 2), uint32_t(i), uint32_t(h), uint32_t(b)), k0, k1);
       const uint32_t us[4] = {u4.x, u4.y, u4.z, u4.w};
+      uint32_t w[4];
+      load4(j0, w);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int j = j0 + q;
-        if (j >= Nkv) break;
-        const uint64_t w = W(j);
         bool keep;
-        uint32_t pq;
-        if (w >= theta) {
+        if (w[q] >= theta) {
           keep = true;  // capped: pi = 1
-          pq = 0;
         } else {
-          const unsigned __int128 X = (unsigned __int128)(R * w) << 32;
-          const unsigned __int128 lhs = (unsigned __int128)(uint64_t(us[q]) + 1ull) * S;
-          keep = (us[q] == 0u) || (lhs <= X);
-          pq = 0;
-          if (keep) {
-            // Pi = max(1, floor(X / S)) < 2^32: double estimate, exact integer fix-up
-            uint64_t est = uint64_t(double(R * w) * 4294967296.0 / double(S));
-            while ((unsigned __int128)est * S > X) --est;
-            while ((unsigned __int128)(est + 1) * S <= X) ++est;
-            pq = est < 1 ? 1u : uint32_t(est);
-          }
+          const uint64_t X = uint64_t(R32) * w[q];
+          keep = us[q] == 0u || mul_le_shift32(us[q], S_hi, S_lo, X);  // (u + 1) S <= X 2^32
         }
-        if (keep) keep_mask |= 1u << q;
-        pis[q] = pq;
+        if (keep && j0 + q < Nkv) keep_mask |= 1u << q;
       }
     }
     // exclusive scan of the per-thread kept counts, in thread (= j) order
@@ -180,14 +203,30 @@ __global__ void __launch_bounds__(256) sip_kernel(const SipArgs a) {
     int pos = base + warp_off + incl - mine;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      if (keep_mask & (1u << q)) {
-        out_idx[pos] = j0 + q;
-        out_pi[pos] = pis[q];
-        ++pos;
-      }
+      if (keep_mask & (1u << q)) out_idx[pos++] = j0 + q;
     }
     base += total;
-    __syncthreads();  // scan[] is reused by the next chunk
+    __syncthreads();  // scan[] is reused by the next chunk; out_idx is read below
+  }
+
+  // ---- inclusion probabilities of the kept entries
+  // Pi = max(1, floor(X 2^32 / S)) < 2^32 for a free entry: a double estimate
+  // (error below one unit), then the exact test a S <= X 2^32 moves it to the
+  // largest such a.
+  const double inv_s32 = S ? 4294967296.0 / double(S) : 0.0;
+  for (int k = tid; k < base; k += kSipThreads) {
+    const int j = out_idx[k];
+    const uint32_t w = kCached ? wcache[j] : quantise_w(__ldg(P + j));
+    uint32_t pq = 0;  // capped: Pi = 2^32
+    if (w < theta) {
+      const uint64_t X = uint64_t(R32) * w;
+      uint64_t est = uint64_t(double(X) * inv_s32);
+      if (est > 0xFFFFFFFFull) est = 0xFFFFFFFFull;
+      while (est > 0 && !mul_le_shift32(uint32_t(est - 1), S_hi, S_lo, X)) --est;
+      while (est < 0xFFFFFFFFull && mul_le_shift32(uint32_t(est), S_hi, S_lo, X)) ++est;
+      pq = est < 1 ? 1u : uint32_t(est);
+    }
+    out_pi[k] = pq;
   }
   if (tid == 0) a.count[row] = base;
 }

@@ -71,34 +71,60 @@ __global__ void __launch_bounds__(256) ksum_kernel(const __nv_bfloat16* __restri
 }
 
 // ----------------------------------------------------------------- k-means
+// Shared memory of one k-means CTA.  The one-hot assignment tile aliases the
+// lo-part centroid tile: the distance product that reads the lo part has
+// completed before the one-hot is written, and the sum product that reads
+// the one-hot has completed before the next lo part is written.  Rows >= C of
+// both stay zero.
 template <int D>
 struct KmSmem {
-  static constexpr int kSlabs = D / 64;
-  static constexpr int kOffQ = 0;                         // 128 x D bf16, SW128 slabs of 16 KB
-  static constexpr int kOffBhi = kOffQ + 2 * 16384;       // 16 x D bf16, SW128 slabs of 2 KB
-  static constexpr int kOffBlo = kOffBhi + 2 * 2048;
-  static constexpr int kOffOneHot = kOffBlo + 2 * 2048;   // 16 clusters x 128 queries bf16, 2 slabs of 2 KB
-  static constexpr int kOffMu = kOffOneHot + 2 * 2048;    // fp32 [16][D]
-  static constexpr int kOffMusq = kOffMu + 16 * D * 4;    // fp32 [16]
-  static constexpr int kOffWcnt = kOffMusq + 64;          // int [4 warps][16]
-  static constexpr int kOffCnt = kOffWcnt + 256;          // int [16]
-  static constexpr int kOffBar = kOffCnt + 64;
+  static constexpr int kOffQ = 0;                      // 128 x 128 bf16, SW128 slabs of 16 KB (slab 1 unused if D = 64)
+  static constexpr int kOffBhi = kOffQ + 2 * 16384;    // 16 x D bf16, SW128 slabs of 2 KB
+  static constexpr int kOffBlo = kOffBhi + 2 * 2048;   // 16 x D bf16 / one-hot 16 x 128 queries
+  static constexpr int kOffMusq = kOffBlo + 2 * 2048;  // float [16][4 warps], partial |mu_c|^2
+  static constexpr int kOffWcnt = kOffMusq + 256;      // int [16][4 warps], partial cluster sizes
+  static constexpr int kOffBar = kOffWcnt + 256;
   static constexpr int kOffMisc = kOffBar + 16;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
 // Element (row, e) of a 128B-swizzled K-major bf16 tile with `slab_bytes`
-// slabs of 64 columns.
-__device__ __forceinline__ float sw_tile_get(const uint8_t* base, int slab_bytes, int row, int e) {
+// slabs of 64 columns: byte offset.
+__device__ __forceinline__ uint32_t sw_tile_off(int slab_bytes, int row, int e) {
   const int slab = e >> 6, col = e & 63;
-  const uint32_t off = uint32_t(slab * slab_bytes) + sw128_offset(uint32_t(row), uint32_t(col >> 3)) +
-                       uint32_t((col & 7) * 2);
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
+  return uint32_t(slab * slab_bytes) + sw128_offset(uint32_t(row), uint32_t(col >> 3)) + uint32_t((col & 7) * 2);
 }
 
-// One CTA (128 threads) per query block.  Per Lloyd iteration, two small
-// tensor-core products:
+// Warp sum of N values per lane (N a power of two <= 32) by recursive halving:
+// lane l returns the total of value (l >> (5 - log2 N)).
+template <int N>
+__device__ __forceinline__ float warp_sum_scatter(const float (&in)[N]) {
+  static_assert(N >= 1 && N <= 32 && (N & (N - 1)) == 0, "N must be a power of two <= 32");
+  const int lane = threadIdx.x & 31;
+  float v[N];
+#pragma unroll
+  for (int k = 0; k < N; ++k) v[k] = in[k];
+  int off = 16;
+#pragma unroll
+  for (int n = N; n > 1; n >>= 1, off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < n / 2; ++k) {
+      const float send = upper ? v[k] : v[k + n / 2];
+      const float keep = upper ? v[k + n / 2] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (; off > 0; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+  return r;
+}
+
+// One CTA (128 threads) per query block.  Thread e < D keeps dimension e of
+// every centroid in registers.  Per Lloyd iteration, two small tensor-core
+// products:
 //   distances  q . mu_c = Q (128 x d) x [mu_hi; mu_lo]^T (d x 16), thread q
 //              reads its 16 columns and takes argmin |mu_c|^2 - 2 q . mu_c;
 //   sums       sum_{q in c} q = Q^T (d x 128) x onehot (128 x 16): Q is read
@@ -107,7 +133,7 @@ __device__ __forceinline__ float sw_tile_get(const uint8_t* base, int slab_bytes
 // Outputs: centroids (fp32, optional), counts (optional), and for the scorer
 // the bf16 centroids and int counts.
 template <int D, int C>
-__global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUtensorMap tmQ, int L, int Nq,
+__global__ void __launch_bounds__(128, C <= 8 ? 5 : 3) kmeans_kernel(const __grid_constant__ CUtensorMap tmQ, int L, int Nq,
                                                      int q_block, int iters, float* __restrict__ cent_out,
                                                      int32_t* __restrict__ counts_out,
                                                      __nv_bfloat16* __restrict__ cent_ws,
@@ -116,10 +142,8 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  float* mu = reinterpret_cast<float*>(smem + SM::kOffMu);
-  float* musq = reinterpret_cast<float*>(smem + SM::kOffMusq);
-  int* wcnt = reinterpret_cast<int*>(smem + SM::kOffWcnt);  // [4][16]
-  int* cnt = reinterpret_cast<int*>(smem + SM::kOffCnt);    // [16]
+  float* musq_part = reinterpret_cast<float*>(smem + SM::kOffMusq);  // [16][4]
+  int* wcnt = reinterpret_cast<int*>(smem + SM::kOffWcnt);           // [16][4]
   const uint32_t bar_q = sbase + SM::kOffBar, bar_mma = sbase + SM::kOffBar + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kOffMisc + 4);
@@ -128,74 +152,66 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
   const int bh = blockIdx.x / Nq;
   const int qi = blockIdx.x - bh * Nq;
   const int n_i = min(q_block, L - qi * q_block);
+  const bool own_dim = tid < D;  // thread e = tid holds dimension e of every centroid
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
     mbar_init(bar_mma, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    mbar_arrive_expect_tx(bar_q, (D / 64) * 16384);
+    for (int s = 0; s < D / 64; ++s)
+      tma_load_3d(sbase + SM::kOffQ + s * 16384, &tmQ, bar_q, s * 64, qi * q_block, bh);
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), 64);  // columns 0-15 distances, 16-31 sums (x32 loads reach 47)
+    tmem_alloc(smem_u32(tmem_slot), 32);  // columns 0-15 distances, 16-31 sums
     tmem_relinquish();
   }
-  // one-hot rows >= C stay zero
-  for (int k = tid; k < 2 * 2048 / 16; k += 128)
-    reinterpret_cast<uint4*>(smem + SM::kOffOneHot)[k] = make_uint4(0, 0, 0, 0);
+  // centroid tiles start zero (rows >= C stay zero)
+  for (int k = tid; k < 2 * 2 * 2048 / 16; k += 128)
+    reinterpret_cast<uint4*>(smem + SM::kOffBhi)[k] = make_uint4(0, 0, 0, 0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tlane = uint32_t(warp * 32) << 16;
 
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bar_q, SM::kSlabs * 16384);
-    for (int s = 0; s < SM::kSlabs; ++s)
-      tma_load_3d(sbase + SM::kOffQ + s * 16384, &tmQ, bar_q, s * 64, qi * q_block, bh);
-  }
   bool ok = mbar_wait(bar_q, 0, abort_flag);
   ok = __syncthreads_and(ok);
 
   const uint8_t* qtile = smem + SM::kOffQ;
-  // initial centroids: query at offset floor((c + 1/2) n_i / C); rows >= C are zero
-  for (int k = tid; k < 16 * D; k += 128) {
-    const int c = k / D, e = k - c * D;
-    float v = 0.f;
-    if (c < C) {
-      const int src = ((2 * c + 1) * n_i) / (2 * C);
-      v = sw_tile_get(qtile, 16384, src, e);
-    }
-    mu[k] = v;
+  // initial centroids: the query at offset floor((c + 1/2) n_i / C)
+  float mu[C];
+  int cnt[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    const int src = ((2 * c + 1) * n_i) / (2 * C);
+    mu[c] = own_dim ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qtile + sw_tile_off(16384, src, tid)))
+                    : 0.f;
+    cnt[c] = 0;
   }
-  __syncthreads();
 
   const uint32_t id_dist = idesc_bf16_f32(128, 16, 0, 0);  // Q (K-major) x mu parts (K-major)
   const uint32_t id_sum = idesc_bf16_f32(128, 16, 1, 0);   // Q^T (MN-major) x onehot (K-major)
   uint32_t phase = 0;
   for (int it = 0; it < iters && ok; ++it) {
-    // centroid tiles (bf16 hi and lo parts, 16 rows, K-major SW128) and |mu|^2
-    for (int k = tid; k < 16 * (D / 8); k += 128) {
-      const int c = k / (D / 8), ch = k - c * (D / 8);  // 8-element chunk
-      uint32_t hi[4], lo[4];
+    // centroid tiles: bf16 hi and lo parts of mu (row c, column e); partial |mu_c|^2
+    float m2[C];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float v0 = mu[c * D + ch * 8 + 2 * h], v1 = mu[c * D + ch * 8 + 2 * h + 1];
-        const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
-        hi[h] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-        lo[h] = pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+    for (int c = 0; c < C; ++c) {
+      m2[c] = mu[c] * mu[c];
+      if (own_dim) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(mu[c]);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(mu[c] - __bfloat162float(hi));
+        const uint32_t off = sw_tile_off(2048, c, tid);
+        *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffBhi + off) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffBlo + off) = lo;
       }
-      const uint32_t off = uint32_t((ch >> 3) * 2048) + sw128_offset(uint32_t(c), uint32_t(ch & 7));
-      *reinterpret_cast<uint4*>(smem + SM::kOffBhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(smem + SM::kOffBlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    if (warp == 0) {
-      for (int c = 0; c < C; ++c) {
-        float s = 0.f;
-        for (int e = lane; e < D; e += 32) s = fmaf(mu[c * D + e], mu[c * D + e], s);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) musq[c] = s;
-      }
+    {
+      const float part = warp_sum_scatter<C>(m2);
+      constexpr int kLanesPer = 32 / C;
+      if ((lane & (kLanesPer - 1)) == 0) musq_part[(lane / kLanesPer) * 4 + warp] = part;
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -219,8 +235,8 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
     if (!ok) break;
     tc_fence_after();
     // dot products of this thread's query with the 16 centroid rows
-    uint32_t dv[32];
-    tmem_ld32(tmem + tlane, dv);
+    uint32_t dv[16];
+    tmem_ld16(tmem + tlane, dv);
     tmem_wait_ld();
     int best = C;  // C marks "no query" (rows beyond the block)
     if (tid < n_i) {
@@ -228,39 +244,33 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
       best = 0;
 #pragma unroll
       for (int c = 0; c < C; ++c) {
-        const float dist = fmaf(-2.f, __uint_as_float(dv[c]), musq[c]);
+        const float4 p4 = *reinterpret_cast<const float4*>(musq_part + 4 * c);
+        const float musq = (p4.x + p4.y) + (p4.z + p4.w);
+        const float dist = fmaf(-2.f, __uint_as_float(dv[c]), musq);
         if (dist < bd) {  // strict: ties go to the lower c
           bd = dist;
           best = c;
         }
       }
     }
-    // cluster sizes (ballots) and this query's one-hot column
+    // cluster sizes (ballots) and this query's one-hot column (over the lo tile)
 #pragma unroll
     for (int c = 0; c < C; ++c) {
       const uint32_t bal = __ballot_sync(0xffffffffu, best == c);
-      if (lane == 0) wcnt[warp * 16 + c] = __popc(bal);
-    }
-    {
-      const int q = tid;
-#pragma unroll
-      for (int c = 0; c < C; ++c) {
-        const uint32_t off = uint32_t((q >> 6) * 2048) + sw128_offset(uint32_t(c), uint32_t((q & 63) >> 3)) +
-                             uint32_t((q & 7) * 2);
-        *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffOneHot + off) =
-            __float2bfloat16_rn(best == c ? 1.f : 0.f);
-      }
+      if (lane == 0) wcnt[4 * c + warp] = __popc(bal);
+      const uint32_t off = uint32_t((tid >> 6) * 2048) + sw128_offset(uint32_t(c), uint32_t((tid & 63) >> 3)) +
+                           uint32_t((tid & 7) * 2);
+      *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffBlo + off) = __float2bfloat16_rn(best == c ? 1.f : 0.f);
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid < C) cnt[tid] = wcnt[tid] + wcnt[16 + tid] + wcnt[32 + tid] + wcnt[48 + tid];
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)  // K = 128 queries, 16 per step
         mma_bf16_ss(tmem + 16u, smem_desc_sw128(sbase + SM::kOffQ + kk * 2048, 16384, 1024),
-                    smem_desc_sw128(sbase + SM::kOffOneHot + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), id_sum,
+                    smem_desc_sw128(sbase + SM::kOffBlo + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), id_sum,
                     kk > 0 ? 1u : 0u);
       mma_commit(bar_mma);
     }
@@ -271,34 +281,36 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
     tc_fence_after();
     // new centroid = sum of members / count (thread e holds dimension e); an
     // empty cluster keeps its centroid
-    uint32_t sv[32];
-    tmem_ld32(tmem + tlane + 16u, sv);
+    uint32_t sv[16];
+    tmem_ld16(tmem + tlane + 16u, sv);
     tmem_wait_ld();
-    if (tid < D) {
 #pragma unroll
-      for (int c = 0; c < C; ++c)
-        if (cnt[c] > 0) mu[c * D + tid] = __uint_as_float(sv[c]) / float(cnt[c]);
+    for (int c = 0; c < C; ++c) {
+      const int4 w4 = *reinterpret_cast<const int4*>(wcnt + 4 * c);
+      cnt[c] = (w4.x + w4.y) + (w4.z + w4.w);
+      if (own_dim && cnt[c] > 0) mu[c] = __uint_as_float(sv[c]) / float(cnt[c]);
     }
-    __syncthreads();
   }
 
   if (ok) {
     const int64_t row0 = (int64_t(bh) * Nq + qi) * C;
-    for (int k = tid; k < C * D; k += 128) {
-      const float v = mu[k];
-      if (cent_out) cent_out[row0 * D + k] = v;
-      cent_ws[row0 * D + k] = __float2bfloat16_rn(v);
-    }
-    if (tid < C) {
-      if (counts_out) counts_out[row0 + tid] = cnt[tid];
-      counts_ws[row0 + tid] = cnt[tid];
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      if (own_dim) {
+        if (cent_out) cent_out[(row0 + c) * D + tid] = mu[c];
+        cent_ws[(row0 + c) * D + tid] = __float2bfloat16_rn(mu[c]);
+      }
+      if (tid == c) {
+        if (counts_out) counts_out[row0 + c] = cnt[c];
+        counts_ws[row0 + c] = cnt[c];
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, 32);
   }
 }
 
