@@ -35,7 +35,8 @@
 // O_1 [256+d, 256+2d); P_s occupies the first 64 columns of S_s.
 // Warps (384 threads, three warpgroups): 0-3 softmax + epilogue of stream 0,
 // 4-7 of stream 1 (warp w owns TMEM lanes 32(w%4)..+31, thread = query row),
-// 8 TMA producer, 9 MMA issuer and TMEM owner, 10-11 idle.  The third
+// 8 TMA producer of Q and K, 9 MMA issuer and TMEM owner, 10 TMA producer
+// of V, 11 idle.  The third
 // warpgroup hands registers to the two softmax warpgroups (setmaxnreg):
 // 384 x 168 at launch = 128 x kRegsCtl + 256 x kRegsSoftmax.  Tiles of the two streams are interleaved in
 // one order ("merged order": 0,1,0,1,... then the longer stream alone) that
@@ -208,15 +209,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
   if (warp >= 8) {
     regs_dec<kRegsCtl>();
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    // Lane e < kSlots owns list slot e of every tile: it reads the list entry
-    // and issues the TMA copies of that KV block's rows into rows
-    // [e*KVB, (e+1)*KVB) of the K tile, and one step later of the V tile.
-    // Lane 0 publishes the slots' weights and valid-key counts with the K tile.
+  if (warp == 8 || warp == 10) {
+    // ----------------------------------------------------------- producers
+    // Warp 8 loads the Q tiles and the K tiles, warp 10 the V tiles: each
+    // walks the merged tile order on its own, so the two TMA streams are
+    // issued independently.  Lane e < kSlots owns list slot e of every tile:
+    // it reads the list entry and issues the TMA copy of that KV block's rows
+    // into rows [e*KVB, (e+1)*KVB) of the tile.  Warp 8's lane 0 publishes the
+    // slots' weights and valid-key counts with the K tile.
+    const bool is_k = warp == 8;
     constexpr uint32_t kTileBytes = uint32_t(SM::kTile);
-    int issued_k[3] = {0, 0, 0}, issued_v[2] = {0, 0}, issued_q[2] = {0, 0};
-    if (lane == 0) {
+    int issued[3] = {0, 0, 0}, issued_q[2] = {0, 0};
+    if (is_k && lane == 0) {
       for (int s = 0; s < 2; ++s) {
         if (T[s] == 0) continue;
         mbar_arrive_expect_tx(bar(kBarQ + s), kTileBytes);
@@ -241,7 +245,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           j = __ldg(a.idx + at);
           pq = __ldg(a.pi_q32 + at);
           if (j < 0 || j >= a.Nkv) {
-            raise_error(AB_ERR_CAPACITY);
+            if (is_k) raise_error(AB_ERR_CAPACITY);
             j = -1;
           }
         }
@@ -251,30 +255,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t pq_cur, pq_next, pq_far;
     fetch(0, j_cur, pq_cur);
     fetch(1, j_next, pq_next);
-    int prev_row = 0, row = 0;
+    const int nstage = is_k ? 3 : 2;
+    const uint32_t full0 = bar(is_k ? kBarKFull : kBarVFull), empty0 = bar(is_k ? kBarKEmpty : kBarVEmpty);
+    const uint32_t dst0 = sbase + (is_k ? SM::kOffK : SM::kOffV);
+    const CUtensorMap* tm = is_k ? &tmK : &tmV;
     bool ok = true;
-    for (int u = 0; u <= G && ok; ++u) {
+    for (int u = 0; u < G; ++u) {
       fetch(u + 2, j_far, pq_far);
-      if (u < G) {
-        int s, t;
-        mg.tile(u, s, t);
-        float bias = 0.f;
-        int valid = 0;
-        if (lane < kSlots) {
-          if (kDense) {
-            row = t * 128;
-            valid = min(128, a.L - row);
-          } else if (j_cur >= 0) {
-            row = j_cur * KVB;
-            valid = min(KVB, a.L - row);
-            bias = pq_cur == 0u ? 0.f : 32.f - log2f(float(pq_cur));  // log2(1/pi), Pi = pq or 2^32
-          } else {
-            row = 0;  // empty slot: any in-range rows (finite data), fully masked
-            valid = 0;
-          }
+      int s, t;
+      mg.tile(u, s, t);
+      float bias = 0.f;
+      int valid = 0, row = 0;  // an empty slot reads any in-range rows (finite data), fully masked
+      if (lane < kSlots) {
+        if (kDense) {
+          row = t * 128;
+          valid = min(128, a.L - row);
+        } else if (j_cur >= 0) {
+          row = j_cur * KVB;
+          valid = min(KVB, a.L - row);
+          bias = pq_cur == 0u ? 0.f : 32.f - log2f(float(pq_cur));  // log2(1/pi), Pi = pq or 2^32
         }
-        const int ks = u % 3;
-        if (!lane0_wait(bar(kBarKEmpty + ks), ((u / 3) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      }
+      const int st = u % nstage, use = u / nstage;
+      const uint32_t full = full0 + 8u * uint32_t(st), empty = empty0 + 8u * uint32_t(st);
+      if (!lane0_wait(empty, (use & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (is_k) {
         float b_all[kSlots];
         int v_all[kSlots];
 #pragma unroll
@@ -283,47 +288,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           v_all[e] = __shfl_sync(0xffffffffu, valid, e);
         }
         if (lane == 0) {
-          float* mb = reinterpret_cast<float*>(smem + SM::kOffMeta + ks * SM::kMetaStride);
-          int* mv = reinterpret_cast<int*>(smem + SM::kOffMeta + ks * SM::kMetaStride + 32);
+          float* mb = reinterpret_cast<float*>(smem + SM::kOffMeta + st * SM::kMetaStride);
+          int* mv = reinterpret_cast<int*>(smem + SM::kOffMeta + st * SM::kMetaStride + 32);
 #pragma unroll
           for (int e = 0; e < kSlots; ++e) {
             mb[e] = b_all[e];
             mv[e] = v_all[e];
           }
-          mbar_arrive_expect_tx(bar(kBarKFull + ks), kTileBytes);
         }
-        __syncwarp();
-        if (lane < kSlots) {
-          if constexpr (kGrouped) {
-            tma_load_5d(sbase + SM::kOffK + ks * SM::kTile + lane * KVB * SM::kSlabs * 128, &tmK,
-                        bar(kBarKFull + ks), 0, 0, 0, row / 8, bh);
-          } else {
-            for (int sl = 0; sl < SM::kSlabs; ++sl)
-              tma_load_3d(sbase + SM::kOffK + ks * SM::kTile + sl * SM::kSlab + lane * KVB * 128, &tmK,
-                          bar(kBarKFull + ks), sl * 64, row, bh);
-          }
-        }
-        issued_k[ks] += 1;
       }
-      if (u >= 1) {
-        const int g = u - 1;
-        const int vs = g & 1;
-        if (!lane0_wait(bar(kBarVEmpty + vs), ((g >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(bar(kBarVFull + vs), kTileBytes);
-        __syncwarp();
-        if (lane < kSlots) {
-          if constexpr (kGrouped) {
-            tma_load_5d(sbase + SM::kOffV + vs * SM::kTile + lane * KVB * SM::kSlabs * 128, &tmV,
-                        bar(kBarVFull + vs), 0, 0, 0, prev_row / 8, bh);
-          } else {
-            for (int sl = 0; sl < SM::kSlabs; ++sl)
-              tma_load_3d(sbase + SM::kOffV + vs * SM::kTile + sl * SM::kSlab + lane * KVB * 128, &tmV,
-                          bar(kBarVFull + vs), sl * 64, prev_row, bh);
-          }
+      if (lane == 0) mbar_arrive_expect_tx(full, kTileBytes);
+      __syncwarp();
+      if (lane < kSlots) {
+        const uint32_t dst = dst0 + uint32_t(st * SM::kTile);
+        if constexpr (kGrouped) {
+          tma_load_5d(dst + lane * KVB * SM::kSlabs * 128, tm, full, 0, 0, 0, row / 8, bh);
+        } else {
+          for (int sl = 0; sl < SM::kSlabs; ++sl)
+            tma_load_3d(dst + sl * SM::kSlab + lane * KVB * 128, tm, full, sl * 64, row, bh);
         }
-        issued_v[vs] += 1;
       }
-      prev_row = row;
+      issued[st] += 1;
       j_cur = j_next;
       pq_cur = pq_next;
       j_next = j_far;
@@ -331,10 +316,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     if (!ok && lane == 0) {
       // let the copies already issued land before shared memory is released
-      for (int k = 0; k < 3; ++k)
-        if (issued_k[k]) mbar_wait_drain(bar(kBarKFull + k), (issued_k[k] - 1) & 1);
-      for (int k = 0; k < 2; ++k)
-        if (issued_v[k]) mbar_wait_drain(bar(kBarVFull + k), (issued_v[k] - 1) & 1);
+      for (int k = 0; k < nstage; ++k)
+        if (issued[k]) mbar_wait_drain(full0 + 8u * uint32_t(k), (issued[k] - 1) & 1);
       for (int s = 0; s < 2; ++s)
         if (issued_q[s]) mbar_wait_drain(bar(kBarQ + s), 0);
     }
