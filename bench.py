@@ -32,13 +32,26 @@ sys.path.insert(0, HERE)
 
 METRIC = "dense-equivalent attention TFLOPS/s + tensor-pipe util; ms per attention layer"
 UNIT = "TFLOP/s"
-WORKLOAD = "wan2.1-14b-480p-self-attention"
+WORKLOAD_NAMES = {"wan480": "wan2.1-14b-480p-self-attention",
+                  "hunyuan720": "hunyuanvideo-720p-self-attention",
+                  "wan720": "wan-720p-self-attention"}
 
 
-def workload(heads=None):
+def workload(args):
+    """The timed layer: Wan2.1-480p by default; the others (and the KV block /
+    keep ratio / C overrides) are for the sweep runs."""
     from block_sparse_attention_queries_b200.synthetic import WORKLOADS
-    w = WORKLOADS["wan480"]
-    return w if not heads else w.with_(H=heads)
+    w = WORKLOADS[getattr(args, "workload", "wan480")]
+    kw = {}
+    if getattr(args, "heads", None):
+        kw["H"] = args.heads
+    if getattr(args, "kv_block", None):
+        kw["kv_block"] = args.kv_block
+    if getattr(args, "keep", None):
+        kw["keep_ratio"] = args.keep
+    if getattr(args, "clusters", None):
+        kw["C"] = args.clusters
+    return w.with_(**kw) if kw else w
 
 
 def dense_flop(w) -> float:
@@ -46,7 +59,7 @@ def dense_flop(w) -> float:
 
 
 def config_dict(w, extra=None):
-    c = {"workload": WORKLOAD, "B": w.B, "H": w.H, "grid_txy": list(w.grid), "L": w.L, "d": w.d,
+    c = {"workload": WORKLOAD_NAMES[w.name], "B": w.B, "H": w.H, "grid_txy": list(w.grid), "L": w.L, "d": w.d,
          "q_block": w.q_block, "kv_block": w.kv_block, "C": w.C, "kmeans_iters": w.kmeans_iters,
          "keep_ratio": w.keep_ratio, "sampler_seed": 42, "data_seed": 1234,
          "l2": "inputs larger than L2 (Q, K, V 335 MB each); no flush"}
@@ -68,64 +81,120 @@ def peaks():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks, power and clock-event reasons sampled during the timed region.
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    Reads NVML (read-only queries) from a background thread every 50 ms; if
+    NVML is unusable it falls back to `nvidia-smi -lms`.  `stop()` returns the
+    summary, or {"error": ...} saying why no sample was taken."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
     def __init__(self, device_index: int):
-        self.proc = None
-        self.path = None
-        try:
-            import torch
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id if hasattr(
-                torch.cuda.get_device_properties(device_index), "pci_bus_id") else None
-        except Exception:
-            bus = None
-        self.id = bus if bus else str(device_index)
+        self.device_index = device_index
+        self.samples = []
+        self.error = None
+        self._stop = None
+        self._thread = None
+        self._smi = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device_index)
+        uuid = str(getattr(props, "uuid", "") or "")
+        if uuid:
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.lower().endswith(uuid.lower()):
+                    return pynvml, h
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
 
     def start(self):
-        import tempfile
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.id}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            nv, h = self._nvml_handle()
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._stop = threading.Event()
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((sm, mx, pw, rs))
+                    except Exception as e:  # keep sampling; report the last failure
+                        self.error = f"nvml: {e}"
+                    self._stop.wait(0.05)
+
+            self._thread = threading.Thread(target=run, daemon=True)
+            self._thread.start()
+            self._nv = nv
+        except Exception as e:
+            self.error = f"nvml unavailable: {e}"
+            self._start_smi()
+
+    def _start_smi(self):
+        import tempfile
+        fd, self._smi_path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        fields = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
+        try:
+            self._smi = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={fields}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self._smi_path, "w"), stderr=subprocess.DEVNULL)
+        except Exception as e:
+            self.error = f"{self.error}; nvidia-smi: {e}"
 
     def wait_first_sample(self, timeout_s: float = 5.0):
         t = time.time()
-        while self.proc is not None and time.time() - t < timeout_s:
-            if os.path.getsize(self.path) > 0:
+        while time.time() - t < timeout_s:
+            if self.samples or (self._smi is not None and os.path.getsize(self._smi_path) > 0):
                 return
-            time.sleep(0.05)
+            if self._thread is None and self._smi is None:
+                return
+            time.sleep(0.02)
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
         rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 7:
-                    rows.append(parts)
-        os.unlink(self.path)
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+            nv = self._nv
+            for sm, mx, pw, rs in self.samples:
+                rows.append((float(sm), float(mx), float(pw),
+                             [name for name, attr in self.REASONS if rs & getattr(nv, attr, 0)]))
+        elif self._smi is not None:
+            self._smi.terminate()
+            try:
+                self._smi.wait(timeout=5)
+            except Exception:
+                self._smi.kill()
+            names = [n for n, _ in self.REASONS[:4]]
+            with open(self._smi_path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    try:
+                        rows.append((float(parts[0]), float(parts[1]), float(parts[2]),
+                                     [names[k] for k in range(4) if parts[3 + k].lower().startswith("active")]))
+                    except (ValueError, IndexError):
+                        continue
+            os.unlink(self._smi_path)
         if not rows:
-            return None
-        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in rows for k in range(4) if r[3 + k].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+            return {"error": self.error or "no samples in the timed region"}
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_median": round(statistics.median(r[2] for r in rows), 1),
+                "reasons": sorted({x for r in rows for x in r[3]}), "samples": len(rows),
+                "source": "nvml" if self._thread is not None else "nvidia-smi"}
 
 
 # ----------------------------------------------------------- our arm (GPU)
@@ -148,7 +217,7 @@ def run_ours(args):
         dist.init_process_group("nccl", rank=rank, world_size=world, device_id=dev,
                                 timeout=datetime.timedelta(seconds=120))
 
-    w = workload(args.heads)
+    w = workload(args)
     p = ab.Params.of(w, seed=42)
     # weak scaling: every rank runs its own layer (independent batch element)
     Qc, Kc, Vc = make_workload_qkv(w, seed=1234 + rank)
@@ -372,7 +441,7 @@ def run_reference(args):
     if rank != 0:
         return None
     from block_sparse_attention_queries_b200.synthetic import make_workload_qkv
-    w = workload(args.heads)
+    w = workload(args)
     Qc, Kc, Vc = make_workload_qkv(w)
     vals = []
     last = None
@@ -399,6 +468,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--heads", type=int, default=None,
                     help="run a smaller case of the same layer with this many heads (profiling only)")
+    ap.add_argument("--workload", choices=["wan480", "hunyuan720", "wan720"], default="wan480",
+                    help="layer shape (default: the Wan2.1-480p headline workload)")
+    ap.add_argument("--kv-block", type=int, default=None, help="KV block size override (sweeps)")
+    ap.add_argument("--keep", type=float, default=None, help="keep ratio override (sweeps)")
+    ap.add_argument("--clusters", type=int, default=None, help="cluster count C override (sweeps)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the end-to-end, dense and CPU-baseline legs (profiling only)")
     args = ap.parse_args()

@@ -77,7 +77,7 @@ struct AttnSmem {
   static constexpr int kOffMeta = kOffV + kVStages * kTile;  // per K stage: 8 biases, 8 valid counts
   static constexpr int kMetaStride = 64;
   static constexpr int kOffBar = kOffMeta + kKStages * kMetaStride;
-  static constexpr int kNumBars = 20;
+  static constexpr int kNumBars = 21;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
@@ -94,6 +94,7 @@ enum : int {
   kBarPFull = 14,  // 2 (per stream, 128 arrivals)
   kBarOFinal = 16, // 2 (per stream)
   kBarDrain = 18,
+  kBarPHalf = 19,  // 2 (per stream, 128 arrivals): keys [0, 64) of P are in TMEM
 };
 
 // Warp-uniform bounded wait: every lane of the calling warp gets the same answer.
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar(kBarVEmpty + s), 1);
       mbar_init(bar(kBarSFull + s), 1);
       mbar_init(bar(kBarPFull + s), 128);
+      mbar_init(bar(kBarPHalf + s), 128);
       mbar_init(bar(kBarOFinal + s), 1);
     }
     for (int k = 0; k < 3; ++k) {
@@ -365,7 +367,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int g = 0; g < G && ok; ++g) {
         int s, t;
         mg.tile(g, s, t);
-        if (!mbar_wait(bar(kBarPFull + s), t & 1, abort_flag)) { ok = false; break; }
+        // P V in two halves of 64 keys: the first starts as soon as the
+        // softmax warps have stored keys [0, 64) of P
+        if (!mbar_wait(bar(kBarPHalf + s), t & 1, abort_flag)) { ok = false; break; }
         if (!mbar_wait(bar(kBarVFull + (g & 1)), (g >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tO = tmem + 256u + uint32_t(s * D);
@@ -376,7 +380,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         vd.lo += uint32_t(g & 1) * uint32_t(SM::kTile >> 4);
         mma_bf16_ts(tO, tP, desc_at(vd, 0), idO, t > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < 8; ++kk) mma_bf16_ts(tO, tP + uint32_t(kk * 8), desc_at(vd, kk * kStepV), idO, 1u);
+        for (int kk = 1; kk < 4; ++kk) mma_bf16_ts(tO, tP + uint32_t(kk * 8), desc_at(vd, kk * kStepV), idO, 1u);
+        if (!mbar_wait(bar(kBarPFull + s), t & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 4; kk < 8; ++kk) mma_bf16_ts(tO, tP + uint32_t(kk * 8), desc_at(vd, kk * kStepV), idO, 1u);
         mma_commit(bar(kBarVEmpty + (g & 1)));
         if (t + 1 < T[s]) {
           ok = issue_S(s, t + 1);
@@ -401,7 +409,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float m_use = -INFINITY;  // reference max (log2 domain)
     float l = 0.f;            // running sum of exp2(x - m_use)
     bool ok = true;
+    // Keys [64h, 64h + 64) of P are stored: let the MMA warp use them.
+    auto publish = [&](int h) {
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar((h == 0 ? kBarPHalf : kBarPFull) + s));
+    };
     for (int t = 0; t < T[s] && ok; ++t) {
+      // O_s is complete up to tile t-1 when S_s(t) is (the commit behind S_s(t)
+      // covers it); a moved reference max rescales it before this tile's P V
+      // product accumulates into it.
+      auto rescale_O = [&](bool need, float alpha) {
+        if (t > 0 && __any_sync(0xffffffffu, need)) {
+          // 8 columns at a time: the scores of this tile are live in registers
+#pragma unroll 1
+          for (int c = 0; c < D / 8; ++c) {
+            uint32_t o[8];
+            tmem_ld8(tO + uint32_t(c * 8), o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st8(tO + uint32_t(c * 8), o);
+          }
+        }
+      };
       const int g = mg.index(s, t);
       const int ks = g % 3;
       if (!warp_wait(bar(kBarSFull + s), t & 1, abort_flag)) { ok = false; break; }
@@ -446,6 +477,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_use = rmax;
           l *= alpha;
         }
+        rescale_O(need, alpha);
         const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
         uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
@@ -467,6 +499,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             pk[k] = pack_bf16x2(p0, p1);
           }
           tmem_st32_ptr(tS + uint32_t(32 * h), pk);
+          publish(h);
         }
         float s0, s1;
         f2_unpack(acc2, s0, s1);
@@ -486,6 +519,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_use = rmax;
           l *= alpha;
         }
+        rescale_O(need, alpha);
         const float mref = (m_use == -INFINITY) ? 0.f : m_use;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -498,24 +532,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             pk[k] = pack_bf16x2(p0, p1);
           }
           tmem_st32_ptr(tS + uint32_t(32 * h), pk);
+          publish(h);
         }
       }
       l += lsum;
-      // O_s is complete up to tile t-1 here (the commit behind S_s(t) covers it)
-      if (t > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + uint32_t(c * 32), o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(tO + uint32_t(c * 32), o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(kBarPFull + s));
     }
     // ---------------------------------------------------------- epilogue
     if (qi < a.Nq) {
