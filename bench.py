@@ -197,6 +197,42 @@ class ClockSampler:
                 "source": "nvml" if self._thread is not None else "nvidia-smi"}
 
 
+# ------------------------------------------------------- ranks (host logic)
+
+def dist_env(gpus: int):
+    """(rank, world, local rank) from the launcher's environment; one process
+    per GPU, so --gpus must equal WORLD_SIZE when more than one rank runs."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and gpus != world:
+        raise SystemExit(f"--gpus {gpus} but WORLD_SIZE {world}")
+    if not 0 <= rank < world:
+        raise SystemExit(f"RANK {rank} outside WORLD_SIZE {world}")
+    return rank, world, local
+
+
+def rank_data_seed(rank: int) -> int:
+    """Each rank runs its own layer: the synthetic inputs are seeded per rank."""
+    return 1234 + rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The slowest rank's time (every rank calls this at the same point)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(w, world: int, ms_step: float) -> float:
+    """Dense-equivalent TFLOP/s of the whole job: every rank processes one layer per step."""
+    return dense_flop(w) * world / (ms_step * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------- our arm (GPU)
 
 def run_ours(args):
@@ -205,11 +241,7 @@ def run_ours(args):
     import block_sparse_attention_queries_b200 as ab
     from block_sparse_attention_queries_b200.synthetic import make_workload_qkv
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.gpus != world and world > 1:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    rank, world, local = dist_env(args.gpus)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -220,7 +252,7 @@ def run_ours(args):
     w = workload(args)
     p = ab.Params.of(w, seed=42)
     # weak scaling: every rank runs its own layer (independent batch element)
-    Qc, Kc, Vc = make_workload_qkv(w, seed=1234 + rank)
+    Qc, Kc, Vc = make_workload_qkv(w, seed=rank_data_seed(rank))
     Q, K, V = (t.to(dev) for t in (Qc, Kc, Vc))
     bufs = ab.Buffers(p, dev)
     stream = torch.cuda.current_stream(dev)
@@ -290,14 +322,9 @@ def run_ours(args):
         exec_flop -= 4.0 * w.d * float((n_i[None, None, :] * part).sum())
     kept_frac = float(cnt.sum()) / (w.B * w.H * w.Nq * w.Nkv)
 
-    # max over ranks
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_step = total_ms / args.steps
-    value = dense_flop(w) * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_value(w, world, ms_step)
     att_avg = statistics.mean(att_ms)
     bf16_peak, hbm_peak, peak_kind = peaks()
     achieved = exec_flop / (att_avg * 1e-3) / 1e12
@@ -437,9 +464,9 @@ def cpu_baseline(w, args, Qc=None, Kc=None, Vc=None):
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
+    rank, _, _ = dist_env(args.gpus)
     if rank != 0:
-        return None
+        return None  # the oracle runs once, on rank 0; the other ranks exit without work
     from block_sparse_attention_queries_b200.synthetic import make_workload_qkv
     w = workload(args)
     Qc, Kc, Vc = make_workload_qkv(w)
