@@ -78,6 +78,29 @@ def peaks():
         return 1590.0, 6650.0, "fallback"
 
 
+# DRAM traffic of one sparse attention launch, from the ncu capture of the
+# 8-head case of the Wan2.1-480p layer (dram__bytes_read.sum +
+# dram__bytes_write.sum = 205.877 MB + 51.283 MB, kv_block 16, 11 % kept),
+# scaled to the layer's heads (the launch's traffic grows with the heads).  It
+# describes the kernel sources it was measured on only: with any other
+# sources (hash below) the bench reports null.
+ATTN_TRAFFIC = {"sources_sha256_16": "421751a677f2f74b", "bytes_per_head": (205.877248e6 + 51.2832e6) / 8,
+                "workload": "wan480", "kv_block": 16, "keep_ratio": 0.11}
+
+
+def attention_traffic(w):
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("ab_attention.cuh", "ab_ptx.cuh"):
+        with open(os.path.join(HERE, "block_sparse_attention_queries_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    t = ATTN_TRAFFIC
+    if (h.hexdigest()[:16] != t["sources_sha256_16"] or w.name != t["workload"] or w.kv_block != t["kv_block"]
+            or abs(w.keep_ratio - t["keep_ratio"]) > 1e-9):
+        return None
+    return round(t["bytes_per_head"] * w.B * w.H)
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -352,7 +375,8 @@ def run_ours(args):
             "speedup_vs_own_dense_kernel": round(dense_ms / ms_step, 3),
             "gpu_launches": 5 * args.steps,
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": bf16_peak, "unit": "TFLOP/s",
-                         "frac": round(achieved / bf16_peak, 4), "traffic": None,
+                         "frac": round(achieved / bf16_peak, 4), "traffic": attention_traffic(w),
+                         "traffic_note": "ncu dram bytes of the 8-head capture x H/8 (profiles/)",
                          "kernel": "ab_attention_kernel<128,16>", "peak_kind": peak_kind,
                          "per_launch_flop": exec_flop},
             "e2e": e2e,
