@@ -314,6 +314,21 @@ __global__ void __launch_bounds__(128, C <= 8 ? 5 : 3) kmeans_kernel(const __gri
   }
 }
 
+// Maximum of v[0 .. N) as a balanced tree of 3-input max operations.
+template <int N>
+__device__ __forceinline__ float max_tree(const float* v) {
+  if constexpr (N == 1) {
+    return v[0];
+  } else if constexpr (N == 2) {
+    return fmaxf(v[0], v[1]);
+  } else if constexpr (N == 3) {
+    return fmax3(v[0], v[1], v[2]);
+  } else {
+    constexpr int kA = N / 3, kB = (N - kA) / 2;
+    return fmax3(max_tree<kA>(v), max_tree<kB>(v + kA), max_tree<N - kA - kB>(v + kA + kB));
+  }
+}
+
 // ------------------------------------------------------------------ scores
 template <int D>
 struct ScSmem {
@@ -462,7 +477,12 @@ __global__ void __launch_bounds__(288, 1)
     const int ch = warp >> 2;  // column half of every chunk
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const float w = roww[r];
+    const float sc = a.scale_log2;
     float* xm = reinterpret_cast<float*>(smem + SM::kOffX);  // [2][2][128]: max, sum per half
+    // Scores are kept in raw units s (x = s * sc); the running max M is in
+    // the x (log2) domain.  Columns past Nkv read as -inf; the last block's
+    // log2(n_last / kv_block) is added to its raw score as bias / sc.
+    const float last_raw = a.last_bias / sc;
     float M = -INFINITY, Z = 0.f;
     bool ok = true;
     for (int g = 0; g < total && ok; ++g) {
@@ -472,6 +492,24 @@ __global__ void __launch_bounds__(288, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + st), (g >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
+      // all 128 columns of this half at once, then release the TMEM buffer
+      float v[128];
+#pragma unroll
+      for (int piece = 0; piece < 4; ++piece)
+        tmem_ld32_nowait(tmem + lane_base + uint32_t(st * 256 + ch * 128 + piece * 32),
+                         reinterpret_cast<uint32_t*>(v) + piece * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kTFree + st));
+      const int j0 = chunk * 256 + ch * 128;
+      if (j0 + 128 > a.Nkv - 1) {  // this half holds the last block or columns past Nkv
+#pragma unroll
+        for (int k = 0; k < 128; ++k) {
+          const int j = j0 + k;
+          v[k] = j < a.Nkv - 1 ? v[k] : (j == a.Nkv - 1 ? v[k] + last_raw : -INFINITY);
+        }
+      }
       if (g == nchunks) {
         // merge the two halves' running max and sum before the second pass
         xm[(0 * 2 + ch) * 128 + r] = M;
@@ -485,52 +523,39 @@ __global__ void __launch_bounds__(288, 1)
         Z = (M == -INFINITY ? 0.f : Z * ex2_approx(M - Mx)) + (M2 == -INFINITY ? 0.f : Z2 * ex2_approx(M2 - Mx));
         M = Mx;
       }
-      const float inv_z = pass2 ? w / Z : 0.f;
-#pragma unroll 1
-      for (int piece = 0; piece < 4; ++piece) {
-        uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + uint32_t(st * 256 + ch * 128 + piece * 32), raw);
-        tmem_wait_ld();
-        const int j0 = chunk * 256 + ch * 128 + piece * 32;
-        float v[32];
+      if (!pass2) {
+        const float pm = fmaxf(M, max_tree<128>(v) * sc);
+        if (pm != -INFINITY) {  // a half entirely past Nkv changes nothing
+          const float nm = -pm;
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const int j = j0 + k;
-          float x = __uint_as_float(raw[k]) * a.scale_log2;
-          if (j == a.Nkv - 1) x += a.last_bias;
-          v[k] = (j < a.Nkv) ? x : -INFINITY;
+          for (int k = 0; k < 128; ++k) s4[k & 3] += ex2_approx(fmaf(v[k], sc, nm));
+          Z = (M == -INFINITY ? 0.f : Z * ex2_approx(M - pm)) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+          M = pm;
         }
-        if (!pass2) {
-          float pm = M;
+      } else {
+        const float inv_z = w / Z;
+        const float nm = -M;
+        constexpr int kPer = 32 / C;
+        const int gl = lane % C;
+        const int i = i0 + r / C;
+        const bool store = i < a.Nq && (r / C) < G;
+        float* prow = a.P + (int64_t(bh) * a.Nq + (store ? i : 0)) * a.Nkv;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) pm = fmaxf(pm, v[k]);
-          if (pm != -INFINITY) {  // a piece entirely past Nkv changes nothing
-            float s = 0.f;
+        for (int piece = 0; piece < 4; ++piece) {
+          float u[32];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) s += ex2_approx(v[k] - pm);
-            Z = (M == -INFINITY ? 0.f : Z * ex2_approx(M - pm)) + s;
-            M = pm;
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = ex2_approx(v[k] - M) * inv_z;
-          group_reduce_scatter<C>(v, lane);
-          constexpr int kPer = 32 / C;
-          const int gl = lane % C;
-          const int i = i0 + r / C;
-          if (i < a.Nq && (r / C) < G) {
-            float* prow = a.P + (int64_t(bh) * a.Nq + i) * a.Nkv;
+          for (int k = 0; k < 32; ++k) u[k] = ex2_approx(fmaf(v[piece * 32 + k], sc, nm)) * inv_z;
+          group_reduce_scatter<C>(u, lane);
+          if (store) {
 #pragma unroll
             for (int k = 0; k < kPer; ++k) {
-              const int j = j0 + gl * kPer + k;
-              if (j < a.Nkv) prow[j] = v[k];
+              const int j = j0 + piece * 32 + gl * kPer + k;
+              if (j < a.Nkv) prow[j] = u[k];
             }
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kTFree + st));
     }
   }
   tc_fence_before();
