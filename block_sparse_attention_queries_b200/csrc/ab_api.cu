@@ -176,7 +176,7 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, floa
   {
     CUtensorMap tmCent, tmKsum;
     if (!make_map(&tmCent, cent_ws, D, uint64_t(d.BH) * d.Nq * d.C, 1, 128)) return AB_ERR_CUDA;
-    if (!make_map(&tmKsum, ksum, D, d.Nkv, d.BH, 256)) return AB_ERR_CUDA;
+    if (!make_map(&tmKsum, ksum, D, d.Nkv, d.BH, 128)) return AB_ERR_CUDA;
     ScoreArgs a{};
     a.L = d.L; a.Nq = d.Nq; a.Nkv = d.Nkv; a.q_block = d.q_block; a.kv_block = d.kv_block;
     a.counts_ws = cnt_ws;

@@ -15,7 +15,7 @@
 //                 argmin per query, then the per-cluster sums as a second
 //                 product Q^T x onehot(assignment) with fp32 accumulation.
 //  score_kernel   S = mu kbar^T / sqrt(d) on the tensor cores for 128/C query
-//                 blocks at once (M = 128 centroid rows, N = 256 KV blocks per
+//                 blocks at once (M = 128 centroid rows, N = 128 KV blocks per
 //                 chunk), per-centroid softmax over j in two passes (max and
 //                 sum, then normalised values), then the cluster-share mixture
 //                 P_ij = sum_c (n_c / n_i) p_cj reduced across the C lanes of
@@ -333,8 +333,8 @@ __device__ __forceinline__ float max_tree(const float* v) {
 template <int D>
 struct ScSmem {
   static constexpr int kSlabs = D / 64;
-  static constexpr int kA = kSlabs * 16384;          // 128 x D bf16
-  static constexpr int kB = kSlabs * 32768;          // 256 x D bf16
+  static constexpr int kA = kSlabs * 16384;          // 128 centroid rows x D bf16
+  static constexpr int kB = kSlabs * 16384;          // 128 K summaries x D bf16 (one chunk)
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kA;           // 2 stages
   static constexpr int kOffW = kOffB + 2 * kB;       // float [128] row weights
@@ -374,11 +374,11 @@ __device__ __forceinline__ void group_reduce_scatter(float (&v)[32], int lane) {
 }
 
 // Warps 0-7 read the scores (warp w: TMEM lanes 32 (w % 4).., columns
-// [128 (w / 4), +128) of every 256-column chunk), warp 8 loads and issues the
-// MMAs.  The two column halves of a row keep separate running max / sum in
+// [64 (w / 4), +64) of every 128-column chunk), warp 8 loads and issues the
+// MMAs.  Two CTAs share an SM (96 KB of shared memory, 256 TMEM columns each).  The two column halves of a row keep separate running max / sum in
 // the first pass and merge them before the second.
 template <int D, int C>
-__global__ void __launch_bounds__(288, 1)
+__global__ void __launch_bounds__(288, 2)
     score_kernel(const __grid_constant__ CUtensorMap tmCent, const __grid_constant__ CUtensorMap tmKsum,
                  const ScoreArgs a) {
   using SM = ScSmem<D>;
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(288, 1)
   const int groups_per_head = (a.Nq + G - 1) / G;
   const int bh = blockIdx.x / groups_per_head;
   const int i0 = (blockIdx.x - bh * groups_per_head) * G;
-  const int nchunks = (a.Nkv + 255) / 256;
+  const int nchunks = (a.Nkv + 127) / 128;
 
   if (tid == 0) {
     mbar_init(bar(kA), 1);
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(288, 1)
     roww[tid] = w;
   }
   if (warp == 8) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -443,13 +443,13 @@ __global__ void __launch_bounds__(288, 1)
         const int chunk = g % nchunks;
         mbar_arrive_expect_tx(bar(kBFull + st), SM::kB);
         for (int s = 0; s < SM::kSlabs; ++s)
-          tma_load_3d(sbase + SM::kOffB + st * SM::kB + s * 32768, &tmKsum, bar(kBFull + st), s * 64,
-                      chunk * 256, bh);
+          tma_load_3d(sbase + SM::kOffB + st * SM::kB + s * 16384, &tmKsum, bar(kBFull + st), s * 64,
+                      chunk * 128, bh);
       };
       load_b(0);
       if (total > 1) load_b(1);
       ok = mbar_wait(bar(kA), 0, abort_flag);
-      const uint32_t idesc = idesc_bf16_f32(128, 256, 0, 0);
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
       for (int g = 0; g < total && ok; ++g) {
         const int st = g & 1;
         if (!mbar_wait(bar(kBFull + st), (g >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -458,8 +458,8 @@ __global__ void __launch_bounds__(288, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t boff = (kk >> 2) * 32768 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + uint32_t(st * 256), smem_desc_sw128(sbase + SM::kOffA + aoff, 16, 1024),
+          const uint32_t boff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + uint32_t(st * 128), smem_desc_sw128(sbase + SM::kOffA + aoff, 16, 1024),
                       smem_desc_sw128(sbase + SM::kOffB + st * SM::kB + boff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(kSFull + st));
@@ -492,20 +492,20 @@ __global__ void __launch_bounds__(288, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + st), (g >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      // all 128 columns of this half at once, then release the TMEM buffer
-      float v[128];
+      // all 64 columns of this half at once, then release the TMEM buffer
+      float v[64];
 #pragma unroll
-      for (int piece = 0; piece < 4; ++piece)
-        tmem_ld32_nowait(tmem + lane_base + uint32_t(st * 256 + ch * 128 + piece * 32),
+      for (int piece = 0; piece < 2; ++piece)
+        tmem_ld32_nowait(tmem + lane_base + uint32_t(st * 128 + ch * 64 + piece * 32),
                          reinterpret_cast<uint32_t*>(v) + piece * 32);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kTFree + st));
-      const int j0 = chunk * 256 + ch * 128;
-      if (j0 + 128 > a.Nkv - 1) {  // this half holds the last block or columns past Nkv
+      const int j0 = chunk * 128 + ch * 64;
+      if (j0 + 64 > a.Nkv - 1) {  // this half holds the last block or columns past Nkv
 #pragma unroll
-        for (int k = 0; k < 128; ++k) {
+        for (int k = 0; k < 64; ++k) {
           const int j = j0 + k;
           v[k] = j < a.Nkv - 1 ? v[k] : (j == a.Nkv - 1 ? v[k] + last_raw : -INFINITY);
         }
@@ -524,28 +524,28 @@ __global__ void __launch_bounds__(288, 1)
         M = Mx;
       }
       if (!pass2) {
-        const float pm = fmaxf(M, max_tree<128>(v) * sc);
+        const float pm = fmaxf(M, max_tree<64>(v) * sc);
         if (pm != -INFINITY) {  // a half entirely past Nkv changes nothing
           const float nm = -pm;
           float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int k = 0; k < 128; ++k) s4[k & 3] += ex2_approx(fmaf(v[k], sc, nm));
+          for (int k = 0; k < 64; ++k) s4[k & 3] += ex2_approx(fmaf(v[k], sc, nm));
           Z = (M == -INFINITY ? 0.f : Z * ex2_approx(M - pm)) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
           M = pm;
         }
       } else {
-        const float inv_z = w / Z;
-        const float nm = -M;
+        // p_cj n_c / n_i = exp2(x - M + log2(w / Z)): the row weight rides in the exponent
+        const float nm = w > 0.f ? __log2f(w / Z) - M : -INFINITY;
         constexpr int kPer = 32 / C;
         const int gl = lane % C;
         const int i = i0 + r / C;
         const bool store = i < a.Nq && (r / C) < G;
         float* prow = a.P + (int64_t(bh) * a.Nq + (store ? i : 0)) * a.Nkv;
 #pragma unroll
-        for (int piece = 0; piece < 4; ++piece) {
+        for (int piece = 0; piece < 2; ++piece) {
           float u[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) u[k] = ex2_approx(fmaf(v[piece * 32 + k], sc, nm)) * inv_z;
+          for (int k = 0; k < 32; ++k) u[k] = ex2_approx(fmaf(v[piece * 32 + k], sc, nm));
           group_reduce_scatter<C>(u, lane);
           if (store) {
 #pragma unroll
@@ -562,7 +562,7 @@ __global__ void __launch_bounds__(288, 1)
   __syncthreads();
   if (warp == 8) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 256);
   }
 }
 
