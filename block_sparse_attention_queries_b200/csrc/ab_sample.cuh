@@ -231,4 +231,122 @@ __global__ void __launch_bounds__(kSipThreads) sip_kernel(const SipArgs a) {
   if (tid == 0) a.count[row] = base;
 }
 
+// One warp per row, for rows of at most 32 * 4 * KMAX blocks: the same
+// arithmetic as sip_kernel (results are identical integers), with the
+// quantised row in registers and warp shuffles instead of block barriers.
+// Lane l owns blocks j = 128 k + 4 l + q (k < KMAX, q < 4), i.e. the same 4
+// consecutive blocks per Philox call.
+template <int KMAX>
+__global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows) {
+  static_assert(KMAX * 4 * 16777216ull < 4294967296ull, "per-lane partial sums must fit 32 bits");
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;  // whole warp: no block-level synchronisation below
+  const int b = row / (a.H * a.Nq);
+  const int h = (row / a.Nq) % a.H;
+  const int i = row % a.Nq;
+  const int Nkv = a.Nkv;
+  const float* P = a.P + int64_t(row) * Nkv;
+  uint32_t w[KMAX][4];
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = 128 * k + 4 * lane + q;
+      w[k][q] = j < Nkv ? quantise_w(__ldg(P + j)) : 0u;  // entries >= Nkv: 0, never capped
+    }
+  }
+
+  // ---- capping threshold (fixed point)
+  uint32_t theta = 0xFFFFFFFFu;
+  uint64_t R = 0, S = 0;
+  for (int round = 0; round <= Nkv + 1; ++round) {
+    uint32_t ncap = 0, part = 0;
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const bool cap = w[k][q] >= theta;
+        ncap += cap ? 1u : 0u;
+        part += cap ? 0u : w[k][q];
+      }
+    }
+    uint64_t sum = part;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ncap += __shfl_xor_sync(0xffffffffu, ncap, o);
+      sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    R = uint64_t(a.Kb) - ncap;
+    S = sum;
+    if (R == 0 || S == 0) break;
+    uint64_t qt = uint64_t(double(S) / double(R));
+    while (qt * R > S) --qt;
+    while ((qt + 1) * R <= S) ++qt;
+    const uint64_t t_new = qt + (qt * R != S ? 1u : 0u);  // ceil(S / R)
+    if (t_new >= theta) break;
+    theta = uint32_t(t_new);
+  }
+
+  // ---- draws and ordered compaction
+  const uint32_t S_hi = uint32_t(S >> 32), S_lo = uint32_t(S);
+  const uint32_t R32 = uint32_t(R);
+  int32_t* out_idx = a.idx + int64_t(row) * Nkv;
+  uint32_t* out_pi = a.pi_q32 + int64_t(row) * Nkv;
+  int base = 0;
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) {
+    if (128 * k >= Nkv) break;  // warp-uniform
+    const int j0 = 128 * k + 4 * lane;
+    uint32_t keep_mask = 0;
+    if (j0 < Nkv) {
+      const uint4 u4 = philox4x32_10(make_uint4(uint32_t(j0 >> 2), uint32_t(i), uint32_t(h), uint32_t(b)),
+                                     a.seed_lo, a.seed_hi);
+      const uint32_t us[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        bool keep;
+        if (w[k][q] >= theta) {
+          keep = true;
+        } else {
+          const uint64_t X = uint64_t(R32) * w[k][q];
+          keep = us[q] == 0u || mul_le_shift32(us[q], S_hi, S_lo, X);
+        }
+        if (keep && j0 + q < Nkv) keep_mask |= 1u << q;
+      }
+    }
+    const int mine = __popc(keep_mask);
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = base + incl - mine;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (keep_mask & (1u << q)) out_idx[pos++] = j0 + q;
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();  // out_idx written by the other lanes is read below
+
+  // ---- inclusion probabilities of the kept entries (as in sip_kernel)
+  const double inv_s32 = S ? 4294967296.0 / double(S) : 0.0;
+  for (int e = lane; e < base; e += 32) {
+    const int j = out_idx[e];
+    const uint32_t wj = quantise_w(__ldg(P + j));
+    uint32_t pq = 0;
+    if (wj < theta) {
+      const uint64_t X = uint64_t(R32) * wj;
+      uint64_t est = uint64_t(double(X) * inv_s32);
+      if (est > 0xFFFFFFFFull) est = 0xFFFFFFFFull;
+      while (est > 0 && !mul_le_shift32(uint32_t(est - 1), S_hi, S_lo, X)) --est;
+      while (est < 0xFFFFFFFFull && mul_le_shift32(uint32_t(est), S_hi, S_lo, X)) ++est;
+      pq = est < 1 ? 1u : uint32_t(est);
+    }
+    out_pi[e] = pq;
+  }
+  if (lane == 0) a.count[row] = base;
+}
+
 }  // namespace ab
