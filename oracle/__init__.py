@@ -58,6 +58,8 @@ def lib():
         L.orc_budget.restype = _ci
         L.orc_sip_row.argtypes = [_f32p, _ci, _ci, _cu64, _ci, _ci, _ci, _i32p, _u32p, _i32p, _vp]
         L.orc_sip_row.restype = _ci
+        L.orc_topk_row.argtypes = [_f32p, _ci, _ci, _i32p, _u32p, _i32p]
+        L.orc_topk_row.restype = _ci
         L.orc_ht_sums.argtypes = [_f32p, _f32p, _f32p, _ci, _ci, _ci, _i32p, _u32p, _ci, _cd,
                                   _f64p, _f64p]
         L.orc_ht_attention_block.argtypes = [_f32p, _f32p, _f32p, _ci, _ci, _ci, _ci, _ci,
@@ -153,6 +155,18 @@ def sip_row(P_row, Kb, seed, b, h, i, want_pi=False):
     n = int(cnt[0])
     out = (idx[:n].copy(), pq[:n].copy(), n)
     return out + (Pi,) if want_pi else out
+
+
+def topk_row(P_row, Kb):
+    """Truncation on one fp32 row: the Kb largest P (ties to the lower j), ascending, pi = 1."""
+    P_row = _f32(P_row)
+    Nkv = P_row.shape[0]
+    idx = np.zeros(Nkv, np.int32)
+    pq = np.zeros(Nkv, np.uint32)
+    cnt = np.zeros(1, np.int32)
+    lib().orc_topk_row(P_row, Nkv, int(Kb), idx, pq, cnt)
+    n = int(cnt[0])
+    return idx[:n].copy(), pq[:n].copy(), n
 
 
 def sip(P, Kb, seed, b_index=None):

@@ -271,6 +271,31 @@ int orc_budget(int Nkv, double keep_ratio) {
 }
 
 // ---------------------------------------------------------------------------
+// Truncation for one query block: the selection that SIP is contrasted with.
+// AB-Attention page, section "Video Difüzyon Modellerinde Dikkat (Attention)
+// Darboğazı" (pruned blocks drop out of the softmax entirely) and section
+// "AB-Attention ve Üç Temel Yeniliği", SIP item (SIP estimates dense attention
+// "instead of truncating it").  Readings: the same IBCS estimate P and the
+// same budget Kb; keep the Kb blocks with the largest P, ties to the lower j;
+// no reweighting (pi = 1, stored as pi_q32 = 0); kept j in ascending order.
+// Returns count = Kb.
+// ---------------------------------------------------------------------------
+int orc_topk_row(const float* P, int Nkv, int Kb, int32_t* idx, uint32_t* pi_q32, int32_t* count) {
+  std::vector<int> order(Nkv);
+  for (int j = 0; j < Nkv; ++j) order[j] = j;
+  // larger P first; equal P: lower j first
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return P[x] > P[y]; });
+  std::vector<int> kept(order.begin(), order.begin() + Kb);
+  std::sort(kept.begin(), kept.end());
+  for (int e = 0; e < Kb; ++e) {
+    idx[e] = kept[e];
+    pi_q32[e] = 0u;
+  }
+  *count = Kb;
+  return Kb;
+}
+
+// ---------------------------------------------------------------------------
 // SIP for one query block (AB-Attention page, "AB-Attention ve Üç Temel
 // Yeniliği", SIP item: blocks are sampled in proportion to the IBCS estimate
 // and the kept ones are reweighted by the inverse inclusion probability).
