@@ -355,11 +355,12 @@ def run_ours(args):
     out = None
     if rank == 0:
         if args.no_extras:
-            e2e, dense_ms, cpu = None, float("nan"), None
+            e2e, dense_ms, cpu, qual = None, float("nan"), None, None
         else:
             # e2e through the public C ABI with host buffers (copies inside the region)
             e2e = run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, max(2, min(args.steps, 5)))
             dense_ms = run_dense(ab, p, Q, K, V, dev, 3)
+            qual = quality(ab, p, Q, K, V, bufs, dev)
             cpu = cpu_baseline(w, args, Qc, Kc, Vc)
         out = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -382,6 +383,7 @@ def run_ours(args):
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk,
+            "quality": qual,
         }
     if world > 1:
         dist.barrier()
@@ -439,6 +441,33 @@ def run_dense(ab, p, Q, K, V, dev, iters):
     t1.record(stream)
     torch.cuda.synchronize(dev)
     return t0.elapsed_time(t1) / iters
+
+
+def quality(ab, p, Q, K, V, bufs, dev):
+    """Information only (no value on the pages pins it): relative L2 distance
+    to dense attention of the SIP output (bufs.O) and of truncation at the same
+    budget (top-Kb blocks of the same P, pi = 1), plus the truncation
+    selection's time."""
+    import torch
+    Od = torch.empty_like(Q)
+    ab.ab_attention_dense(p, Q, K, V, out=Od)
+    idx, piq, cnt = ab.ab_sample_topk(p, bufs.P)
+    stream = torch.cuda.current_stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(3):
+        ab.ab_sample_topk(p, bufs.P)
+    t1.record(stream)
+    Ot = ab.ab_attention(p, Q, K, V, idx, piq, cnt)
+    torch.cuda.synchronize(dev)
+    ref = torch.linalg.vector_norm(Od.double())
+
+    def rel(o):
+        return round(float(torch.linalg.vector_norm(o.double() - Od.double()) / ref), 5)
+
+    return {"rel_l2_sip_vs_dense": rel(bufs.O), "rel_l2_truncation_vs_dense": rel(Ot),
+            "ms_sample_truncation": round(t0.elapsed_time(t1) / 3, 4),
+            "note": "same P and budget; information only, not a gate"}
 
 
 # ---------------------------------------------------------- CPU oracle arm

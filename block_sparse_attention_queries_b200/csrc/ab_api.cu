@@ -352,6 +352,20 @@ ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* 
   return do_sample(d, P, idx, pi_q32, count, static_cast<cudaStream_t>(stream));
 }
 
+ab_status ab_sample_topk(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,
+                         void* stream) {
+  Dims d;
+  const ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  if (!P || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
+  if (!aligned16(P) || !aligned16(idx) || !aligned16(pi_q32) || !aligned16(count)) return AB_ERR_INVALID_ARG;
+  SipArgs a{};
+  a.P = P; a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
+  a.H = d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
+  topk_kernel<<<unsigned(d.BH * d.Nq), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
+}
+
 ab_status ab_attention(const ab_params* p, const void* Q, const void* K, const void* V, const int32_t* idx,
                        const uint32_t* pi_q32, const int32_t* count, void* O, void* stream) {
   Dims d;

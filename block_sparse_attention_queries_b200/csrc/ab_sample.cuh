@@ -349,4 +349,118 @@ __global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows
   if (lane == 0) a.count[row] = base;
 }
 
+// Truncation, the selection SIP is contrasted with (AB-Attention page,
+// section "Video Difüzyon Modellerinde Dikkat (Attention) Darboğazı": pruned
+// blocks drop out of the softmax; SIP item: SIP estimates dense attention
+// "instead of truncating it").  One CTA (256 threads) per row keeps the Kb
+// blocks with the largest P, ties to the lower j, in ascending order, with
+// pi = 1 (pi_q32 = 0).  P >= 0, so the order of the values is the order of
+// their bit patterns as unsigned integers: a 4-pass, 8-bit radix select finds
+// the Kb-th largest key T and how many keys equal to T are kept; one ordered
+// pass then writes every key > T and the first of the keys == T.
+__global__ void __launch_bounds__(256) topk_kernel(const SipArgs a) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t sel[2];
+  __shared__ uint32_t scan[8];
+  const int row = blockIdx.x;
+  const float* P = a.P + int64_t(row) * a.Nkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Nkv = a.Nkv;
+  uint32_t prefix = 0, pmask = 0, need = uint32_t(a.Kb);  // rank of T among the keys matching prefix
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    hist[tid] = 0;
+    __syncthreads();
+    for (int j = tid; j < Nkv; j += 256) {
+      const uint32_t key = __float_as_uint(__ldg(P + j));
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds bins 255 - 8 l - t (t = 0..7), i.e. the bins in descending order
+      uint32_t c[8], tot = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        c[t] = hist[255 - 8 * lane - t];
+        tot += c[t];
+      }
+      uint32_t incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t above = incl - tot;  // keys in higher bins
+      if (above < need && need <= incl) {  // exactly one lane: T's digit is in its bins
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (above < need && need <= above + c[t]) {
+            sel[0] = uint32_t(255 - 8 * lane - t);
+            sel[1] = need - above;
+          }
+          above += c[t];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= sel[0] << shift;
+    pmask |= 0xFFu << shift;
+    need = sel[1];
+    __syncthreads();  // hist and sel are rewritten by the next pass
+  }
+  const uint32_t T = prefix;
+  const uint32_t take_eq = need;  // keys equal to T that are kept (the lowest j)
+
+  // ordered pass: 4 consecutive j per thread per 1024-wide chunk
+  int32_t* out_idx = a.idx + int64_t(row) * Nkv;
+  uint32_t* out_pi = a.pi_q32 + int64_t(row) * Nkv;
+  uint32_t base_gt = 0, base_eq = 0;
+  for (int c0 = 0; c0 < Nkv; c0 += 1024) {
+    const int j0 = c0 + 4 * tid;
+    uint32_t gt = 0, eq = 0;  // 4-bit masks
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (j0 + q < Nkv) {
+        const uint32_t key = __float_as_uint(__ldg(P + j0 + q));
+        gt |= (key > T ? 1u : 0u) << q;
+        eq |= (key == T ? 1u : 0u) << q;
+      }
+    }
+    // exclusive scan of packed (gt count, eq count), 16 bits each (<= 1024 per chunk)
+    const uint32_t mine = uint32_t(__popc(gt)) | (uint32_t(__popc(eq)) << 16);
+    uint32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) scan[warp] = incl;
+    __syncthreads();
+    uint32_t woff = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const uint32_t v = scan[w];
+      if (w < warp) woff += v;
+      total += v;
+    }
+    const uint32_t excl = woff + incl - mine;
+    uint32_t n_gt = base_gt + (excl & 0xFFFFu), n_eq = base_eq + (excl >> 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const bool is_gt = (gt >> q) & 1u, is_eq = (eq >> q) & 1u;
+      if (is_gt || (is_eq && n_eq < take_eq)) {
+        const uint32_t pos = n_gt + (n_eq < take_eq ? n_eq : take_eq);
+        out_idx[pos] = j0 + q;
+        out_pi[pos] = 0u;
+      }
+      n_gt += is_gt ? 1u : 0u;
+      n_eq += is_eq ? 1u : 0u;
+    }
+    base_gt += total & 0xFFFFu;
+    base_eq += total >> 16;
+    __syncthreads();  // scan[] is reused by the next chunk
+  }
+  if (tid == 0) a.count[row] = a.Kb;
+}
+
 }  // namespace ab

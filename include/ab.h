@@ -13,7 +13,8 @@
  *                 every KV block's share of the block's attention mass.
  *   ab_sample     SIP, sampling with inclusion-probability weighting: draw KV
  *                 blocks in proportion to that estimate and keep each kept
- *                 block's inverse inclusion probability.
+ *                 block's inverse inclusion probability.  (ab_sample_topk is
+ *                 the truncation it replaces, for comparison.)
  *   ab_attention  the kernel that packs the small kept KV blocks into full
  *                 tensor-core tiles and computes the 1/pi-weighted softmax, an
  *                 estimate of softmax(Q K^T / sqrt(d)) V (the formula of the
@@ -138,6 +139,20 @@ ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* 
                     void* stream);
 
 /*
+ * Truncation, the selection SIP replaces (AB-Attention page, section "Video
+ * Difüzyon Modellerinde Dikkat (Attention) Darboğazı": pruned blocks vanish
+ * from the softmax; SIP item: SIP estimates dense attention "instead of
+ * truncating it").  For every row of P, keep the Kb blocks with the largest
+ * P (Kb as for ab_sample; ties to the lower block index), in ascending order,
+ * with weight 1 (pi_q32 = 0); count = Kb.  Same arguments, layout, ownership
+ * and errors as ab_sample; P must be >= 0 (as ab_select writes it).  With
+ * ab_attention this is block-sparse attention without reweighting, at the same
+ * budget as SIP.
+ */
+ab_status ab_sample_topk(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,
+                         void* stream);
+
+/*
  * 1/pi-weighted block-sparse attention (AB-Attention page, SIP item: one pass
  * estimates dense attention instead of truncating it; "Donanım Dostu Çekirdek"
  * item: KV blocks much smaller than a tile are packed into full tensor-core
@@ -146,7 +161,7 @@ ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* 
  *   O_q = sum_{j in list(i)} w_j sum_{k in j, k < L} e^{s_k} v_k
  *       / sum_{j in list(i)} w_j sum_{k in j, k < L} e^{s_k};
  * a query block with count 0 gets O = 0.  The lists may come from ab_sample
- * or from any other source; they must be ascending or not, but each entry must
+ * (or ab_sample_topk) or from any other source, in any order; each entry must
  * satisfy 0 <= idx < Nkv and count <= Nkv (violations raise AB_ERR_CAPACITY on
  * the device and the offending entries or rows are skipped).
  *
