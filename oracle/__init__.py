@@ -59,6 +59,10 @@ def lib():
         L.orc_sip_row.argtypes = [_f32p, _ci, _ci, _cu64, _ci, _ci, _ci, _i32p, _u32p, _i32p, _vp]
         L.orc_sip_row.restype = _ci
         L.orc_topk_row.argtypes = [_f32p, _ci, _ci, _i32p, _u32p, _i32p]
+        L.orc_systematic_row.argtypes = [_f32p, _ci, _ci, _cu64, _ci, _ci, _ci, _i32p, _u32p, _i32p]
+        L.orc_systematic_row.restype = _ci
+        L.orc_systematic_row_u.argtypes = [_f32p, _ci, _ci, _cu64, _i32p, _u32p, _i32p]
+        L.orc_systematic_row_u.restype = _ci
         L.orc_topk_row.restype = _ci
         L.orc_ht_sums.argtypes = [_f32p, _f32p, _f32p, _ci, _ci, _ci, _i32p, _u32p, _ci, _cd,
                                   _f64p, _f64p]
@@ -155,6 +159,30 @@ def sip_row(P_row, Kb, seed, b, h, i, want_pi=False):
     n = int(cnt[0])
     out = (idx[:n].copy(), pq[:n].copy(), n)
     return out + (Pi,) if want_pi else out
+
+
+def systematic_row(P_row, Kb, seed, b, h, i):
+    """Systematic sampling with SIP's inclusion probabilities on one fp32 row: idx, pi_q32, count."""
+    P_row = _f32(P_row)
+    Nkv = P_row.shape[0]
+    idx = np.zeros(Nkv, np.int32)
+    pq = np.zeros(Nkv, np.uint32)
+    cnt = np.zeros(1, np.int32)
+    lib().orc_systematic_row(P_row, Nkv, int(Kb), ctypes.c_uint64(int(seed)), b, h, i, idx, pq, cnt)
+    n = int(cnt[0])
+    return idx[:n].copy(), pq[:n].copy(), n
+
+
+def systematic_row_u(P_row, Kb, U):
+    """The systematic selection for an explicit offset U in [0, 2^32)."""
+    P_row = _f32(P_row)
+    Nkv = P_row.shape[0]
+    idx = np.zeros(Nkv, np.int32)
+    pq = np.zeros(Nkv, np.uint32)
+    cnt = np.zeros(1, np.int32)
+    lib().orc_systematic_row_u(P_row, Nkv, int(Kb), ctypes.c_uint64(int(U)), idx, pq, cnt)
+    n = int(cnt[0])
+    return idx[:n].copy(), pq[:n].copy(), n
 
 
 def topk_row(P_row, Kb):

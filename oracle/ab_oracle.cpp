@@ -314,8 +314,8 @@ int orc_topk_row(const float* P, int Nkv, int Kb, int32_t* idx, uint32_t* pi_q32
 // P is one fp32 row [Nkv]; idx and pi_q32 hold up to Nkv entries.  Pi (may be
 // null) receives every Pi_j as a 64-bit integer.  Returns count.
 // ---------------------------------------------------------------------------
-int orc_sip_row(const float* P, int Nkv, int Kb, uint64_t seed, int b, int h, int i,
-                int32_t* idx, uint32_t* pi_q32, int32_t* count, uint64_t* Pi) {
+// Steps 1-2 of SIP: the Q32 inclusion probabilities Pi_j of one row.
+static void sip_probabilities(const float* P, int Nkv, int Kb, uint64_t* Pi) {
   std::vector<uint64_t> W(Nkv);
   for (int j = 0; j < Nkv; ++j) {
     const double scaled = std::floor((double)P[j] * 16777216.0);
@@ -340,17 +340,25 @@ int orc_sip_row(const float* P, int Nkv, int Kb, uint64_t seed, int b, int h, in
     }
     if (!grew) break;
   }
+  for (int j = 0; j < Nkv; ++j) {
+    if (capped[j]) {
+      Pi[j] = 1ull << 32;
+    } else {
+      const unsigned __int128 num = ((unsigned __int128)R * W[j]) << 32;
+      uint64_t pij = (uint64_t)(num / S);
+      Pi[j] = pij < 1 ? 1 : pij;
+    }
+  }
+}
+
+int orc_sip_row(const float* P, int Nkv, int Kb, uint64_t seed, int b, int h, int i,
+                int32_t* idx, uint32_t* pi_q32, int32_t* count, uint64_t* Pi) {
+  std::vector<uint64_t> pis(Nkv);
+  sip_probabilities(P, Nkv, Kb, pis.data());
   const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
   int n = 0;
   for (int j = 0; j < Nkv; ++j) {
-    uint64_t pij;
-    if (capped[j]) {
-      pij = 1ull << 32;
-    } else {
-      const unsigned __int128 num = ((unsigned __int128)R * W[j]) << 32;
-      pij = (uint64_t)(num / S);
-      if (pij < 1) pij = 1;
-    }
+    const uint64_t pij = pis[j];
     if (Pi) Pi[j] = pij;
     const uint32_t ctr[4] = {(uint32_t)(j >> 2), (uint32_t)i, (uint32_t)h, (uint32_t)b};
     uint32_t u4[4];
@@ -364,6 +372,51 @@ int orc_sip_row(const float* P, int Nkv, int Kb, uint64_t seed, int b, int h, in
   }
   *count = n;
   return n;
+}
+
+// ---------------------------------------------------------------------------
+// Systematic sampling with the same inclusion probabilities: the sampling
+// design is not fixed by the pages (AB-Attention page, SIP item: blocks are
+// sampled in proportion to the IBCS estimate and reweighted by the inverse
+// inclusion probability).  Reading: one uniform offset U per row, word 0 of
+// Philox4x32-10 with counter (0xFFFFFFFF, i, h, b) (outside the per-block
+// counters j div 4 of SIP), key (seed lo, seed hi); with C_j = sum_{k<j} Pi_k,
+// block j is kept iff one of the points U + m 2^32 (m = 0, 1, ...) lies in
+// [C_j, C_j + Pi_j).  Each block is kept with probability Pi_j / 2^32 (so
+// the same 1/pi weights make numerator and denominator unbiased) and the
+// sample size is fixed up to one: the number of points below sum_j Pi_j.
+// Lists as for SIP (ascending, pi_q32 = Pi mod 2^32).  Returns count.
+// ---------------------------------------------------------------------------
+// The selection for a given offset U in [0, 2^32) (U is a parameter so that
+// tests can sweep it).
+int orc_systematic_row_u(const float* P, int Nkv, int Kb, uint64_t U, int32_t* idx, uint32_t* pi_q32,
+                         int32_t* count) {
+  std::vector<uint64_t> pis(Nkv);
+  sip_probabilities(P, Nkv, Kb, pis.data());
+  // points strictly below x: U + m 2^32 < x for m >= 0
+  auto points_below = [&](uint64_t x) -> uint64_t { return x > U ? ((x - U - 1) >> 32) + 1 : 0; };
+  uint64_t C = 0;
+  int n = 0;
+  for (int j = 0; j < Nkv; ++j) {
+    const uint64_t next = C + pis[j];
+    if (points_below(next) - points_below(C) == 1) {
+      idx[n] = j;
+      pi_q32[n] = (uint32_t)(pis[j] & 0xffffffffull);
+      n += 1;
+    }
+    C = next;
+  }
+  *count = n;
+  return n;
+}
+
+int orc_systematic_row(const float* P, int Nkv, int Kb, uint64_t seed, int b, int h, int i,
+                       int32_t* idx, uint32_t* pi_q32, int32_t* count) {
+  const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  const uint32_t ctr[4] = {0xFFFFFFFFu, (uint32_t)i, (uint32_t)h, (uint32_t)b};
+  uint32_t u4[4];
+  philox_10(ctr, key, u4);
+  return orc_systematic_row_u(P, Nkv, Kb, (uint64_t)u4[0], idx, pi_q32, count);
 }
 
 // ---------------------------------------------------------------------------
