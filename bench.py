@@ -459,13 +459,22 @@ def quality(ab, p, Q, K, V, bufs, dev):
         ab.ab_sample_topk(p, bufs.P)
     t1.record(stream)
     Ot = ab.ab_attention(p, Q, K, V, idx, piq, cnt)
+    sidx, spiq, scnt = ab.ab_sample_systematic(p, bufs.P)
+    t2, t3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t2.record(stream)
+    for _ in range(3):
+        ab.ab_sample_systematic(p, bufs.P)
+    t3.record(stream)
+    Os = ab.ab_attention(p, Q, K, V, sidx, spiq, scnt)
     torch.cuda.synchronize(dev)
     ref = torch.linalg.vector_norm(Od.double())
 
     def rel(o):
         return round(float(torch.linalg.vector_norm(o.double() - Od.double()) / ref), 5)
 
-    return {"rel_l2_sip_vs_dense": rel(bufs.O), "rel_l2_truncation_vs_dense": rel(Ot),
+    return {"rel_l2_sip_vs_dense": rel(bufs.O), "rel_l2_systematic_vs_dense": rel(Os),
+            "rel_l2_truncation_vs_dense": rel(Ot),
+            "ms_sample_systematic": round(t2.elapsed_time(t3) / 3, 4),
             "ms_sample_truncation": round(t0.elapsed_time(t1) / 3, 4),
             "note": "same P and budget; information only, not a gate"}
 

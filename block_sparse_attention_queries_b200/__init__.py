@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "AB_OK", 1: "AB_ERR_INVALID_ARG", 2: "AB_ERR_UNSUPPORTED", 3:
                 4: "AB_ERR_CAPACITY", 5: "AB_ERR_TIMEOUT", 6: "AB_ERR_WORKSPACE"}
 
 # every symbol include/ab.h declares
-EXPORTS = ("ab_budget", "ab_workspace_size", "ab_select", "ab_sample", "ab_sample_topk", "ab_attention",
+EXPORTS = ("ab_budget", "ab_workspace_size", "ab_select", "ab_sample", "ab_sample_systematic", "ab_sample_topk", "ab_attention",
            "ab_attention_dense", "ab_forward", "ab_forward_host", "ab_get_device_error",
            "ab_status_string", "ab_select_static")
 
@@ -97,6 +97,7 @@ def lib(path: str = LIB_PATH):
         L.ab_select.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ab_sample.argtypes = [P, vp, vp, vp, vp, vp]
         L.ab_sample_topk.argtypes = [P, vp, vp, vp, vp, vp]
+        L.ab_sample_systematic.argtypes = [P, vp, vp, vp, vp, vp]
         L.ab_attention.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp]
         L.ab_attention_dense.argtypes = [P, vp, vp, vp, vp, vp]
         L.ab_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -105,7 +106,8 @@ def lib(path: str = LIB_PATH):
         L.ab_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
         L.ab_status_string.argtypes = [ctypes.c_int]
         L.ab_status_string.restype = ctypes.c_char_p
-        for name in ("ab_workspace_size", "ab_select", "ab_sample", "ab_sample_topk", "ab_attention", "ab_attention_dense",
+        for name in ("ab_workspace_size", "ab_select", "ab_sample", "ab_sample_systematic", "ab_sample_topk", "ab_attention",
+                     "ab_attention_dense",
                      "ab_forward", "ab_forward_host", "ab_get_device_error", "ab_select_static"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -192,6 +194,24 @@ def ab_sample(p: Params, P):
     _check(lib().ab_sample(ctypes.byref(p.c()), _ptr(P), _ptr(idx), _ptr(piq), _ptr(cnt), _stream(dev)),
            "ab_sample")
     return idx, piq, cnt
+
+
+def _lists_call(fn_name, p: Params, P):
+    import torch
+    if P.dtype != torch.float32 or tuple(P.shape) != (p.B, p.H, p.Nq, p.Nkv) or not P.is_contiguous():
+        raise ValueError("P must be contiguous fp32 [B,H,Nq,Nkv]")
+    dev = P.device
+    idx = torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev)
+    piq = torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev)
+    cnt = torch.zeros(p.B, p.H, p.Nq, dtype=torch.int32, device=dev)
+    _check(getattr(lib(), fn_name)(ctypes.byref(p.c()), _ptr(P), _ptr(idx), _ptr(piq), _ptr(cnt), _stream(dev)),
+           fn_name)
+    return idx, piq, cnt
+
+
+def ab_sample_systematic(p: Params, P):
+    """Systematic sampling with SIP's inclusion probabilities: same outputs as ab_sample."""
+    return _lists_call("ab_sample_systematic", p, P)
 
 
 def ab_sample_topk(p: Params, P):

@@ -273,11 +273,11 @@ ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q3
   } else if (d.Nkv <= kSipSmemCap) {
     const int smem = 16 * ((d.Nkv + 3) / 4);
     if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(sip_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        cudaFuncSetAttribute(sip_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return AB_ERR_CUDA;
-    sip_kernel<true><<<unsigned(d.BH * d.Nq), kSipThreads, smem, st>>>(a);
+    sip_kernel<true, false><<<unsigned(d.BH * d.Nq), kSipThreads, smem, st>>>(a);
   } else {
-    sip_kernel<false><<<unsigned(d.BH * d.Nq), kSipThreads, 0, st>>>(a);
+    sip_kernel<false, false><<<unsigned(d.BH * d.Nq), kSipThreads, 0, st>>>(a);
   }
   return launch_status();
 }
@@ -350,6 +350,30 @@ ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* 
   const ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   return do_sample(d, P, idx, pi_q32, count, static_cast<cudaStream_t>(stream));
+}
+
+ab_status ab_sample_systematic(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,
+                               void* stream) {
+  Dims d;
+  const ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  if (!P || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
+  if (!aligned16(P) || !aligned16(idx) || !aligned16(pi_q32) || !aligned16(count)) return AB_ERR_INVALID_ARG;
+  SipArgs a{};
+  a.P = P; a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
+  a.H = d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
+  a.seed_lo = uint32_t(d.seed); a.seed_hi = uint32_t(d.seed >> 32);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d.Nkv <= kSipSmemCap) {
+    const int smem = 16 * ((d.Nkv + 3) / 4);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(sip_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return AB_ERR_CUDA;
+    sip_kernel<true, true><<<unsigned(d.BH * d.Nq), kSipThreads, smem, st>>>(a);
+  } else {
+    sip_kernel<false, true><<<unsigned(d.BH * d.Nq), kSipThreads, 0, st>>>(a);
+  }
+  return launch_status();
 }
 
 ab_status ab_sample_topk(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,

@@ -72,12 +72,116 @@ __device__ __forceinline__ bool mul_le_shift32(uint32_t a_minus_1, uint32_t S_hi
   return r >= (1ull << 32) || t <= (r << 32);
 }
 
+// Pi = max(1, floor(X 2^32 / S)) < 2^32 for a free block (X = R W < S): a
+// double estimate (error below one unit), then the exact test a S <= X 2^32
+// moves it to the largest such a.
+__device__ __forceinline__ uint32_t pi_free(uint64_t X, uint32_t S_hi, uint32_t S_lo, double inv_s32) {
+  uint64_t est = uint64_t(double(X) * inv_s32);
+  if (est > 0xFFFFFFFFull) est = 0xFFFFFFFFull;
+  while (est > 0 && !mul_le_shift32(uint32_t(est - 1), S_hi, S_lo, X)) --est;
+  while (est < 0xFFFFFFFFull && mul_le_shift32(uint32_t(est), S_hi, S_lo, X)) ++est;
+  return est < 1 ? 1u : uint32_t(est);
+}
+
 constexpr int kSipThreads = 256;
 constexpr int kSipSmemCap = 16384;  // entries of W cached in shared memory (64 KB)
 
-template <bool kCached>
+// Systematic sampling with the same inclusion probabilities (the sampling
+// design is left open by the pages; SIP item of the AB-Attention page): one
+// offset U per row, word 0 of Philox4x32-10 at counter (0xFFFFFFFF, i, h, b);
+// with C_j the cumulative Pi in block order, block j is kept iff a point
+// U + m 2^32 (m >= 0) lies in [C_j, C_j + Pi_j).  Each block is kept with
+// probability Pi_j / 2^32; the sample size is floor or ceil of sum Pi / 2^32.
+// A block-wide scan of the 64-bit Pi gives C_j; a second scan places the kept
+// blocks in ascending order.
+template <typename Load4>
+__device__ __forceinline__ void systematic_pass(const SipArgs& a, uint32_t theta, uint64_t R, uint64_t S, int b,
+                                                int h, int i, Load4 load4, uint64_t* scan64, int* scan) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = blockIdx.x;
+  const int Nkv = a.Nkv;
+  const uint32_t S_hi = uint32_t(S >> 32), S_lo = uint32_t(S);
+  const uint32_t R32 = uint32_t(R);
+  const double inv_s32 = S ? 4294967296.0 / double(S) : 0.0;
+  const uint64_t U = philox4x32_10(make_uint4(0xFFFFFFFFu, uint32_t(i), uint32_t(h), uint32_t(b)), a.seed_lo,
+                                   a.seed_hi).x;
+  auto points_below = [&](uint64_t x) -> uint64_t { return x > U ? ((x - U - 1) >> 32) + 1 : 0; };
+  int32_t* out_idx = a.idx + int64_t(row) * Nkv;
+  uint32_t* out_pi = a.pi_q32 + int64_t(row) * Nkv;
+  uint64_t base_c = 0;
+  int base = 0;
+  for (int c0 = 0; c0 < Nkv; c0 += 4 * kSipThreads) {
+    const int j0 = c0 + 4 * tid;
+    uint64_t pis[4] = {0, 0, 0, 0};
+    if (j0 < Nkv) {
+      uint32_t w[4];
+      load4(j0, w);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (j0 + q < Nkv) pis[q] = w[q] >= theta ? (1ull << 32) : uint64_t(pi_free(uint64_t(R32) * w[q], S_hi, S_lo, inv_s32));
+    }
+    // exclusive block scan of the per-thread Pi sums
+    const uint64_t mine = (pis[0] + pis[1]) + (pis[2] + pis[3]);
+    uint64_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) scan64[warp] = incl;
+    __syncthreads();
+    uint64_t woff = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const uint64_t v = scan64[w];
+      if (w < warp) woff += v;
+      total += v;
+    }
+    uint64_t C = base_c + woff + incl - mine;
+    uint32_t keep_mask = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint64_t next = C + pis[q];
+      if (j0 + q < Nkv && points_below(next) - points_below(C) == 1) keep_mask |= 1u << q;
+      C = next;
+    }
+    // ordered positions of the kept blocks
+    const int kept = __popc(keep_mask);
+    int kincl = kept;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, kincl, o);
+      if (lane >= o) kincl += y;
+    }
+    if (lane == 31) scan[warp] = kincl;
+    __syncthreads();
+    int kwoff = 0, ktotal = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const int v = scan[w];
+      if (w < warp) kwoff += v;
+      ktotal += v;
+    }
+    int pos = base + kwoff + kincl - kept;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (keep_mask & (1u << q)) {
+        out_idx[pos] = j0 + q;
+        out_pi[pos] = uint32_t(pis[q] & 0xFFFFFFFFull);
+        ++pos;
+      }
+    }
+    base_c += total;
+    base += ktotal;
+    __syncthreads();  // scan64[] and scan[] are reused by the next chunk
+  }
+  if (tid == 0) a.count[row] = base;
+}
+
+template <bool kCached, bool kSystematic>
 __global__ void __launch_bounds__(kSipThreads) sip_kernel(const SipArgs a) {
   __shared__ uint64_t red_sum[2][8];
+  __shared__ uint64_t scan64[8];
   __shared__ uint32_t red_cnt[2][8];
   __shared__ int scan[8];
   extern __shared__ uint4 wcache4[];  // [ceil(Nkv / 4)] when cached; entries >= Nkv hold 0
@@ -156,6 +260,10 @@ __global__ void __launch_bounds__(kSipThreads) sip_kernel(const SipArgs a) {
     theta = uint32_t(t_new);  // t_new < theta <= 2^32 - 1
   }
 
+  if constexpr (kSystematic) {
+    systematic_pass(a, theta, R, S, b, h, i, load4, scan64, scan);
+    return;
+  }
   // ---- draws and ordered compaction, 4 consecutive j per thread per chunk
   const uint32_t k0 = a.seed_lo, k1 = a.seed_hi;
   const uint32_t S_hi = uint32_t(S >> 32), S_lo = uint32_t(S);
@@ -217,16 +325,7 @@ __global__ void __launch_bounds__(kSipThreads) sip_kernel(const SipArgs a) {
   for (int k = tid; k < base; k += kSipThreads) {
     const int j = out_idx[k];
     const uint32_t w = kCached ? wcache[j] : quantise_w(__ldg(P + j));
-    uint32_t pq = 0;  // capped: Pi = 2^32
-    if (w < theta) {
-      const uint64_t X = uint64_t(R32) * w;
-      uint64_t est = uint64_t(double(X) * inv_s32);
-      if (est > 0xFFFFFFFFull) est = 0xFFFFFFFFull;
-      while (est > 0 && !mul_le_shift32(uint32_t(est - 1), S_hi, S_lo, X)) --est;
-      while (est < 0xFFFFFFFFull && mul_le_shift32(uint32_t(est), S_hi, S_lo, X)) ++est;
-      pq = est < 1 ? 1u : uint32_t(est);
-    }
-    out_pi[k] = pq;
+    out_pi[k] = w < theta ? pi_free(uint64_t(R32) * w, S_hi, S_lo, inv_s32) : 0u;  // capped: Pi = 2^32
   }
   if (tid == 0) a.count[row] = base;
 }
@@ -335,16 +434,7 @@ __global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows
   for (int e = lane; e < base; e += 32) {
     const int j = out_idx[e];
     const uint32_t wj = quantise_w(__ldg(P + j));
-    uint32_t pq = 0;
-    if (wj < theta) {
-      const uint64_t X = uint64_t(R32) * wj;
-      uint64_t est = uint64_t(double(X) * inv_s32);
-      if (est > 0xFFFFFFFFull) est = 0xFFFFFFFFull;
-      while (est > 0 && !mul_le_shift32(uint32_t(est - 1), S_hi, S_lo, X)) --est;
-      while (est < 0xFFFFFFFFull && mul_le_shift32(uint32_t(est), S_hi, S_lo, X)) ++est;
-      pq = est < 1 ? 1u : uint32_t(est);
-    }
-    out_pi[e] = pq;
+    out_pi[e] = wj < theta ? pi_free(uint64_t(R32) * wj, S_hi, S_lo, inv_s32) : 0u;
   }
   if (lane == 0) a.count[row] = base;
 }

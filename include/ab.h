@@ -13,8 +13,9 @@
  *                 every KV block's share of the block's attention mass.
  *   ab_sample     SIP, sampling with inclusion-probability weighting: draw KV
  *                 blocks in proportion to that estimate and keep each kept
- *                 block's inverse inclusion probability.  (ab_sample_topk is
- *                 the truncation it replaces, for comparison.)
+ *                 block's inverse inclusion probability.  (ab_sample_systematic
+ *                 draws a fixed-size sample with the same probabilities;
+ *                 ab_sample_topk is the truncation SIP replaces.)
  *   ab_attention  the kernel that packs the small kept KV blocks into full
  *                 tensor-core tiles and computes the 1/pi-weighted softmax, an
  *                 estimate of softmax(Q K^T / sqrt(d)) V (the formula of the
@@ -139,6 +140,23 @@ ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* 
                     void* stream);
 
 /*
+ * Systematic sampling with SIP's inclusion probabilities: a fixed-size
+ * alternative to ab_sample's independent draws (AB-Attention page, SIP item:
+ * blocks are sampled in proportion to the IBCS estimate and reweighted by the
+ * inverse inclusion probability; the sampling design is left open).  Pi_j as
+ * for ab_sample; one offset U per row, word 0 of Philox4x32-10 at counter
+ * (0xFFFFFFFF, i, h, b) with key (seed lo, seed hi); with C_j the sum of Pi_k
+ * over k < j, block j is kept iff some point U + m 2^32 (m >= 0) lies in
+ * [C_j, C_j + Pi_j).  Every block is kept with probability Pi_j / 2^32 (the
+ * same weights make numerator and denominator unbiased) and count is floor or
+ * ceil of sum_j Pi_j / 2^32 (Kb or Kb - 1).  Same arguments, layout,
+ * ownership and errors as ab_sample; results are bit-identical to this
+ * integer specification.
+ */
+ab_status ab_sample_systematic(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,
+                               void* stream);
+
+/*
  * Truncation, the selection SIP replaces (AB-Attention page, section "Video
  * Difüzyon Modellerinde Dikkat (Attention) Darboğazı": pruned blocks vanish
  * from the softmax; SIP item: SIP estimates dense attention "instead of
@@ -161,7 +179,8 @@ ab_status ab_sample_topk(const ab_params* p, const float* P, int32_t* idx, uint3
  *   O_q = sum_{j in list(i)} w_j sum_{k in j, k < L} e^{s_k} v_k
  *       / sum_{j in list(i)} w_j sum_{k in j, k < L} e^{s_k};
  * a query block with count 0 gets O = 0.  The lists may come from ab_sample
- * (or ab_sample_topk) or from any other source, in any order; each entry must
+ * (ab_sample_systematic, ab_sample_topk) or from any other source, in any
+ * order; each entry must
  * satisfy 0 <= idx < Nkv and count <= Nkv (violations raise AB_ERR_CAPACITY on
  * the device and the offending entries or rows are skipped).
  *

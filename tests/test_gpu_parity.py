@@ -227,6 +227,46 @@ def test_truncated_attention_small_workload(dev):
     assert_close_attention(np32(O), ref, "truncated small")
 
 
+@pytest.mark.parametrize("B,H,L,kvb,keep,seed", [(2, 3, 1000, 16, 0.1, 42), (1, 2, 4096, 16, 0.5, 7),
+                                                 (2, 1, 8192, 32, 0.05, 2**63 + 12345),
+                                                 (1, 1, 2000, 64, 1.0, 3), (1, 2, 118800, 16, 0.08, 42),
+                                                 (1, 1, 262400, 16, 0.02, 5)])
+def test_sample_systematic_bit_exact(dev, B, H, L, kvb, keep, seed):
+    p = ab.Params(B=B, H=H, L=L, d=128, q_block=128, kv_block=kvb, C=8, keep_ratio=keep, seed=seed)
+    Nq = min(p.Nq, 12) if L > 100000 else p.Nq
+    P = _skewed_P(B, H, p.Nq, p.Nkv, seed % 1000)
+    idx, piq, cnt = ab.ab_sample_systematic(p, torch.from_numpy(P).to(dev))
+    torch.cuda.synchronize()
+    _no_device_error(dev)
+    gi, gp, gc = _lists_np(idx, piq, cnt)
+    Kb = oracle.budget(p.Nkv, keep)
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nq):
+                oi, op, on = oracle.systematic_row(P[b, h, i], Kb, seed, b, h, i)
+                assert gc[b, h, i] == on and Kb - 1 <= on <= Kb
+                np.testing.assert_array_equal(gi[b, h, i, :on], oi)
+                np.testing.assert_array_equal(gp[b, h, i, :on], op)
+
+
+def test_systematic_attention_small_workload(dev):
+    # ab_select -> ab_sample_systematic -> ab_attention against the oracle
+    w = WORKLOADS["small"]
+    p = ab.Params.of(w)
+    Qc, Kc, Vc = make_workload_qkv(w)
+    Q, K, V = (t.to(dev) for t in (Qc, Kc, Vc))
+    P = ab.ab_select(p, Q, K)
+    idx, piq, cnt = ab.ab_sample_systematic(p, P)
+    O = ab.ab_attention(p, Q, K, V, idx, piq, cnt)
+    torch.cuda.synchronize()
+    _no_device_error(dev)
+    gi, gp, gc = _lists_np(idx, piq, cnt)
+    units = _all_units(p)
+    Qn, Kn, Vn = np32(Qc), np32(Kc), np32(Vc)
+    ref = _stack_units(p, oracle_ht_units(Qn, Kn, Vn, p.q_block, p.kv_block, units, gi, gp, gc), units)
+    assert_close_attention(np32(O), ref, "systematic small")
+
+
 def test_philox_word3_matches_curand_device():
     # cuRAND's device Philox4x32_10 (a library routine) vs the oracle on
     # counters with all four words populated.
