@@ -2,6 +2,7 @@
 // checks, workspace layout, TMA descriptors and kernel launches.  The library
 // allocates no memory; every buffer belongs to the caller.
 #include <cmath>
+#include <vector>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -260,13 +261,17 @@ ab_status do_select(const Dims& d, const void* Q, const void* K, float* P, float
   return d.d == 128 ? run_select<128>(d, Q, K, P, cent, counts, w, st) : run_select<64>(d, Q, K, P, cent, counts, w, st);
 }
 
-ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count, cudaStream_t st) {
+// rows: the rows of this call (d.BH * d.Nq unless a caller processes a range of
+// heads); H and row0 place them in the full problem for the draws' counters.
+ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count, cudaStream_t st,
+                    int H = -1, int64_t row0 = 0) {
   if (!P || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
   if (!aligned16(P) || !aligned16(idx) || !aligned16(pi_q32) || !aligned16(count)) return AB_ERR_INVALID_ARG;
   SipArgs a{};
   a.P = P; a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
-  a.H = d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
+  a.H = H > 0 ? H : d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
   a.seed_lo = uint32_t(d.seed); a.seed_hi = uint32_t(d.seed >> 32);
+  a.row0 = row0;
   const int rows = d.BH * d.Nq;
   if (d.Nkv <= 2048) {  // one warp per row, the row in registers
     sip_warp_kernel<16><<<unsigned((rows + 7) / 8), 256, 0, st>>>(a, rows);
@@ -420,22 +425,98 @@ ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const voi
   return do_attention(d, Q, K, V, idx, pi_q32, count, O, false, st);
 }
 
+namespace {
+
+// Streams and events of one pipelined host call, released on every path.
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  std::vector<cudaEvent_t> ev;
+  ~HostPipe() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);  // released once their work completes
+    if (in) cudaStreamDestroy(in);
+    if (out) cudaStreamDestroy(out);
+  }
+  bool event(cudaEvent_t* e) {
+    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    ev.push_back(*e);
+    return true;
+  }
+};
+
+}  // namespace
+
 ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_host, const void* V_host,
                           void* O_host, void* Q, void* K, void* V, float* P, int32_t* idx, uint32_t* pi_q32,
                           int32_t* count, void* O, void* workspace, size_t ws_bytes, void* stream) {
   Dims d;
   ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
-  if (!Q_host || !K_host || !V_host || !O_host || !Q || !K || !V || !O) return AB_ERR_INVALID_ARG;
+  if (!Q_host || !K_host || !V_host || !O_host || !Q || !K || !V || !O || !idx || !pi_q32 || !count)
+    return AB_ERR_INVALID_ARG;
   if (ws_bytes < workspace_layout(d).total) return AB_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t bytes = size_t(d.BH) * d.L * d.d * 2;
-  if (cudaMemcpyAsync(Q, Q_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
-  if (cudaMemcpyAsync(K, K_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
-  if (cudaMemcpyAsync(V, V_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
-  s = ab_forward(p, Q, K, V, P, idx, pi_q32, count, O, workspace, ws_bytes, stream);
-  if (s != AB_OK) return s;
-  if (cudaMemcpyAsync(O_host, O, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return AB_ERR_CUDA;
+  const size_t head_bytes = size_t(d.L) * d.d * 2;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return AB_ERR_CUDA;
+  // groups of up to ceil(BH / 5) heads, a multiple of 4 so that every group's
+  // row offset keeps the per-row buffers 16-byte aligned
+  const int per = (((d.BH + 4) / 5) + 3) / 4 * 4;
+  if (cap != cudaStreamCaptureStatusNone || per >= d.BH) {  // one stream: copies, path, copy back
+    const size_t bytes = size_t(d.BH) * head_bytes;
+    if (cudaMemcpyAsync(Q, Q_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
+    if (cudaMemcpyAsync(K, K_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
+    if (cudaMemcpyAsync(V, V_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
+    s = ab_forward(p, Q, K, V, P, idx, pi_q32, count, O, workspace, ws_bytes, stream);
+    if (s != AB_OK) return s;
+    if (cudaMemcpyAsync(O_host, O, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return AB_ERR_CUDA;
+    return AB_OK;
+  }
+  // Pipelined over groups of heads (every (b, h) is independent): the inputs
+  // of group c + 1 cross PCIe while group c computes on the caller's stream
+  // and group c - 1's output crosses back, on two streams of this call.
+  HostPipe pipe;
+  if (cudaStreamCreateWithFlags(&pipe.in, cudaStreamNonBlocking) != cudaSuccess) return AB_ERR_CUDA;
+  if (cudaStreamCreateWithFlags(&pipe.out, cudaStreamNonBlocking) != cudaSuccess) return AB_ERR_CUDA;
+  cudaEvent_t start, done;
+  if (!pipe.event(&start) || !pipe.event(&done)) return AB_ERR_CUDA;
+  if (cudaEventRecord(start, st) != cudaSuccess) return AB_ERR_CUDA;  // after the caller's earlier work
+  if (cudaStreamWaitEvent(pipe.in, start, 0) != cudaSuccess) return AB_ERR_CUDA;
+  if (cudaStreamWaitEvent(pipe.out, start, 0) != cudaSuccess) return AB_ERR_CUDA;
+  auto bf = [](const void* base, size_t off) { return static_cast<const uint8_t*>(base) + off; };
+  auto bw = [](void* base, size_t off) { return static_cast<uint8_t*>(base) + off; };
+  for (int bh0 = 0; bh0 < d.BH; bh0 += per) {
+    const int nbh = per < d.BH - bh0 ? per : d.BH - bh0;
+    const size_t off = size_t(bh0) * head_bytes, bytes = size_t(nbh) * head_bytes;
+    cudaEvent_t in_done, comp_done;
+    if (!pipe.event(&in_done) || !pipe.event(&comp_done)) return AB_ERR_CUDA;
+    if (cudaMemcpyAsync(bw(Q, off), bf(Q_host, off), bytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess ||
+        cudaMemcpyAsync(bw(K, off), bf(K_host, off), bytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess ||
+        cudaMemcpyAsync(bw(V, off), bf(V_host, off), bytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess)
+      return AB_ERR_CUDA;
+    if (cudaEventRecord(in_done, pipe.in) != cudaSuccess) return AB_ERR_CUDA;
+    if (cudaStreamWaitEvent(st, in_done, 0) != cudaSuccess) return AB_ERR_CUDA;
+    // the group as a problem of its own (B = 1, H = nbh); the draws keep the
+    // counters of the full problem (H, first row)
+    Dims dc = d;
+    dc.B = 1; dc.H = nbh; dc.BH = nbh;
+    const size_t rows0 = size_t(bh0) * d.Nq;
+    float* Pc = P + rows0 * d.Nkv;
+    int32_t* idxc = idx + rows0 * d.Nkv;
+    uint32_t* pic = pi_q32 + rows0 * d.Nkv;
+    int32_t* cntc = count + rows0;
+    s = do_select(dc, bf(Q, off), bf(K, off), Pc, nullptr, nullptr, workspace, ws_bytes, st);
+    if (s != AB_OK) return s;
+    s = do_sample(dc, Pc, idxc, pic, cntc, st, d.H, int64_t(rows0));
+    if (s != AB_OK) return s;
+    s = do_attention(dc, bf(Q, off), bf(K, off), bf(V, off), idxc, pic, cntc, bw(O, off), false, st);
+    if (s != AB_OK) return s;
+    if (cudaEventRecord(comp_done, st) != cudaSuccess) return AB_ERR_CUDA;
+    if (cudaStreamWaitEvent(pipe.out, comp_done, 0) != cudaSuccess) return AB_ERR_CUDA;
+    if (cudaMemcpyAsync(bw(O_host, off), bf(O, off), bytes, cudaMemcpyDeviceToHost, pipe.out) != cudaSuccess)
+      return AB_ERR_CUDA;
+  }
+  if (cudaEventRecord(done, pipe.out) != cudaSuccess) return AB_ERR_CUDA;
+  if (cudaStreamWaitEvent(st, done, 0) != cudaSuccess) return AB_ERR_CUDA;  // the caller's stream covers it all
   return AB_OK;
 }
 

@@ -54,6 +54,7 @@ struct SipArgs {
   int32_t* count;
   int H, Nq, Nkv, Kb;
   uint32_t seed_lo, seed_hi;
+  int64_t row0;  // global index of the first row (for the draws' counters): rows are (b, h, i) in order
 };
 
 __device__ __forceinline__ uint32_t quantise_w(float p) {
@@ -187,9 +188,10 @@ __global__ void __launch_bounds__(kSipThreads) sip_kernel(const SipArgs a) {
   extern __shared__ uint4 wcache4[];  // [ceil(Nkv / 4)] when cached; entries >= Nkv hold 0
   uint32_t* wcache = reinterpret_cast<uint32_t*>(wcache4);
   const int row = blockIdx.x;
-  const int b = row / (a.H * a.Nq);
-  const int h = (row / a.Nq) % a.H;
-  const int i = row % a.Nq;
+  const int64_t grow = a.row0 + row;
+  const int b = int(grow / (int64_t(a.H) * a.Nq));
+  const int h = int((grow / a.Nq) % a.H);
+  const int i = int(grow % a.Nq);
   const float* P = a.P + int64_t(row) * a.Nkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Nkv = a.Nkv;
@@ -341,9 +343,10 @@ __global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;  // whole warp: no block-level synchronisation below
-  const int b = row / (a.H * a.Nq);
-  const int h = (row / a.Nq) % a.H;
-  const int i = row % a.Nq;
+  const int64_t grow = a.row0 + row;
+  const int b = int(grow / (int64_t(a.H) * a.Nq));
+  const int h = int((grow / a.Nq) % a.H);
+  const int i = int(grow % a.Nq);
   const int Nkv = a.Nkv;
   const float* P = a.P + int64_t(row) * Nkv;
   uint32_t w[KMAX][4];

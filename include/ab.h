@@ -212,9 +212,16 @@ ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const voi
 /*
  * ab_forward from HOST buffers: copies Q_host, K_host, V_host (host, [B, H, L,
  * d] bf16; page-locked memory gives asynchronous copies) to the device buffers
- * Q, K, V, runs ab_forward, and copies O back to O_host (host, [B, H, L, d]
- * bf16).  All copies are enqueued on `stream`; O_host is valid once the stream
- * has been synchronised.  The device buffers are owned by the caller.
+ * Q, K, V, runs the path, and copies O back to O_host (host, [B, H, L, d]
+ * bf16).  Results are bit-identical to ab_forward on the same inputs.  When
+ * B * H > 4 and `stream` is not being captured, the call pipelines groups of
+ * heads (every (b, h) is independent): the inputs of one group cross PCIe on
+ * an internal stream while the previous group computes on `stream` and the
+ * one before it copies back on a second internal stream; the two streams and
+ * their events are created by the call and released when its work completes,
+ * and `stream` waits for all of it.  Otherwise everything is enqueued on
+ * `stream`.  O_host is valid once `stream` has been synchronised.  The device
+ * buffers are owned by the caller.
  */
 ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_host, const void* V_host,
                           void* O_host, void* Q, void* K, void* V, float* P, int32_t* idx,

@@ -372,6 +372,29 @@ def test_small_workload_end_to_end(dev):
         np.testing.assert_array_equal(gi[r][:gc[r]], sg[r][0])
 
 
+@pytest.mark.parametrize("B,H,grid", [(2, 3, (2, 16, 16)), (1, 9, (2, 12, 20)), (1, 2, (2, 16, 16))])
+def test_forward_host_equals_device_path(dev, B, H, grid):
+    # ab_forward_host (pinned host buffers in and out; head groups pipelined
+    # over PCIe when B*H > 4) gives the device path's lists and output bit for bit
+    L = grid[0] * grid[1] * grid[2]
+    p = ab.Params(B=B, H=H, L=L, d=128, q_block=128, kv_block=16, C=8, keep_ratio=0.15, seed=99)
+    (Qc, Kc, Vc), (Q, K, V), _ = _inputs(p, grid, 8, 13, dev)
+    ref = ab.ab_forward(p, Q, K, V)
+    torch.cuda.synchronize()
+    Qh, Kh, Vh = (t.pin_memory() for t in (Qc, Kc, Vc))
+    Oh = torch.empty_like(Qc).pin_memory()
+    Qd, Kd, Vd = (torch.empty_like(t) for t in (Q, K, V))
+    bufs = ab.Buffers(p, dev)
+    ab.ab_forward_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, bufs, dev)
+    torch.cuda.synchronize()
+    _no_device_error(dev)
+    assert torch.equal(bufs.count, ref.count)
+    assert torch.equal(bufs.idx, ref.idx)
+    assert torch.equal(bufs.pi_q32, ref.pi_q32)
+    assert torch.equal(bufs.O, ref.O)
+    assert torch.equal(Oh, ref.O.cpu())
+
+
 @pytest.mark.parametrize("d,kvb", [(128, 16), (64, 32), (128, 64)])
 def test_full_budget_equals_dense_bitwise(dev, d, kvb):
     grid = (4, 18, 20)  # L = 1440: ragged last query block and last KV block for 64
