@@ -458,9 +458,9 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
   const size_t head_bytes = size_t(d.L) * d.d * 2;
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return AB_ERR_CUDA;
-  // groups of up to ceil(BH / 5) heads, a multiple of 4 so that every group's
+  // groups of up to ceil(BH / 10) heads, a multiple of 4 so that every group's
   // row offset keeps the per-row buffers 16-byte aligned
-  const int per = (((d.BH + 4) / 5) + 3) / 4 * 4;
+  const int per = (((d.BH + 9) / 10) + 3) / 4 * 4;
   if (cap != cudaStreamCaptureStatusNone || per >= d.BH) {  // one stream: copies, path, copy back
     const size_t bytes = size_t(d.BH) * head_bytes;
     if (cudaMemcpyAsync(Q, Q_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
