@@ -532,6 +532,8 @@ def run_reference(args):
     from block_sparse_attention_queries_b200.synthetic import make_workload_qkv
     w = workload(args)
     Qc, Kc, Vc = make_workload_qkv(w)
+    for _ in range(args.warmup):  # untimed warm-up steps
+        cpu_baseline(w, args, Qc, Kc, Vc)
     vals = []
     last = None
     for _ in range(args.steps):
