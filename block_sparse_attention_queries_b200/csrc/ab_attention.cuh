@@ -32,15 +32,17 @@
 // also guarantees that O_s(t) is complete when the softmax reads S_s(t+1).
 //
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d),
-// O_1 [256+d, 256+2d); P_s occupies the first 64 columns of S_s.
+// O_1 [256+d, 256+2d); P_s (bf16 pairs) occupies the first 64 columns of S_s.
+// P is stored in two halves of 64 keys, each announced on its own barrier,
+// so that the P V product starts on the first half.
 // Warps (384 threads, three warpgroups): 0-3 softmax + epilogue of stream 0,
 // 4-7 of stream 1 (warp w owns TMEM lanes 32(w%4)..+31, thread = query row),
-// 8 TMA producer of Q and K, 9 MMA issuer and TMEM owner, 10 TMA producer
-// of V, 11 idle.  The third
-// warpgroup hands registers to the two softmax warpgroups (setmaxnreg):
-// 384 x 168 at launch = 128 x kRegsCtl + 256 x kRegsSoftmax.  Tiles of the two streams are interleaved in
-// one order ("merged order": 0,1,0,1,... then the longer stream alone) that
-// the producer, the MMA warp and the K / V rings share.
+// 8 TMA producer of Q and K, 9 MMA issuer and TMEM owner, 10 TMA producer of
+// V, 11 idle.  The third warpgroup hands registers to the two softmax
+// warpgroups (setmaxnreg): 384 x 168 at launch = 128 x kRegsCtl + 256 x
+// kRegsSoftmax.  Tiles of the two streams are interleaved in one order
+// ("merged order": 0,1,0,1,... then the longer stream alone) that the
+// producers, the MMA warp and the K / V rings share.
 #pragma once
 
 #include "ab_ptx.cuh"
