@@ -34,7 +34,9 @@
  *    the runs of kv_block tokens (Nkv = ceil(L / kv_block)); the last block of
  *    each kind may be partial.
  *  - Memory: the caller allocates and owns every buffer (device memory unless a
- *    call says "host"); the library allocates nothing and frees nothing.
+ *    call says "host"); the library allocates and frees no memory (only a
+ *    pipelined ab_forward_host call creates, and releases, two streams and
+ *    their events).
  *    Every device pointer must be 16-byte aligned.
  *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  *    Every call only enqueues work on it and returns; results are ready when
