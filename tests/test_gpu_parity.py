@@ -372,6 +372,32 @@ def test_small_workload_end_to_end(dev):
         np.testing.assert_array_equal(gi[r][:gc[r]], sg[r][0])
 
 
+@pytest.mark.parametrize("L,qb,kvb,C", [(1, 64, 16, 1), (5, 128, 16, 4), (17, 64, 16, 16), (130, 128, 64, 2),
+                                         (257, 128, 32, 8)])
+def test_tiny_sequences_end_to_end(dev, L, qb, kvb, C):
+    # degenerate sizes: a single token, one partial KV block, fewer queries
+    # than clusters, a ragged last query block of 1-2 rows
+    p = ab.Params(B=1, H=2, L=L, d=64, q_block=qb, kv_block=kvb, C=C, keep_ratio=0.3, seed=5)
+    grid = (1, 1, L)
+    (Qc, Kc, Vc), (Q, K, V), (Qn, Kn, Vn) = _inputs(p, grid, 8, 21, dev)
+    bufs = ab.ab_forward(p, Q, K, V)
+    torch.cuda.synchronize()
+    _no_device_error(dev)
+    gi, gp, gc = _lists_np(bufs.idx, bufs.pi_q32, bufs.count)
+    Kb = oracle.budget(p.Nkv, p.keep_ratio)
+    units = _all_units(p)
+    sg = oracle_sip_rows(bufs.P.cpu().numpy(), Kb, p.seed, units)
+    for r in units:
+        assert gc[r] == sg[r][2]
+        np.testing.assert_array_equal(gi[r][:gc[r]], sg[r][0])
+    ref = _stack_units(p, oracle_ht_units(Qn, Kn, Vn, p.q_block, p.kv_block, units, gi, gp, gc), units)
+    assert_close_attention(np32(bufs.O), ref, f"tiny L={L}")
+    Od = ab.ab_attention_dense(p, Q, K, V)
+    torch.cuda.synchronize()
+    refd = _stack_units(p, oracle_dense_units(Qn, Kn, Vn, p.q_block, units), units)
+    assert_close_attention(np32(Od), refd, f"tiny dense L={L}")
+
+
 @pytest.mark.parametrize("B,H,grid", [(2, 3, (2, 16, 16)), (1, 9, (2, 12, 20)), (1, 2, (2, 16, 16))])
 def test_forward_host_equals_device_path(dev, B, H, grid):
     # ab_forward_host (pinned host buffers in and out; head groups pipelined
