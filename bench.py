@@ -352,13 +352,14 @@ def run_ours(args):
     bf16_peak, hbm_peak, peak_kind = peaks()
     achieved = exec_flop / (att_avg * 1e-3) / 1e12
 
+    # e2e through the public C ABI with host buffers (copies inside the region), on every rank
+    e2e = None if args.no_extras else run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, max(2, min(args.steps, 5)),
+                                              world, barrier)
     out = None
     if rank == 0:
         if args.no_extras:
-            e2e, dense_ms, cpu, qual = None, float("nan"), None, None
+            dense_ms, cpu, qual = float("nan"), None, None
         else:
-            # e2e through the public C ABI with host buffers (copies inside the region)
-            e2e = run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, max(2, min(args.steps, 5)))
             dense_ms = run_dense(ab, p, Q, K, V, dev, 3)
             qual = quality(ab, p, Q, K, V, bufs, dev)
             cpu = cpu_baseline(w, args, Qc, Kc, Vc)
@@ -407,13 +408,17 @@ def _sample(ab, p, bufs):
                             ab._ptr(bufs.count), st), "ab_sample")
 
 
-def run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, steps):
+def run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, steps, world=1, barrier=None):
+    """The same metric through the public host-buffer call, every rank on its
+    own layer; the time is the slowest rank's, the bytes the whole job's."""
     import torch
     Qh, Kh, Vh = (t.pin_memory() for t in (Qc, Kc, Vc))
     Oh = torch.empty_like(Qc).pin_memory()
     Qd, Kd, Vd = (torch.empty_like(Qc, device=dev) for _ in range(3))
     stream = torch.cuda.current_stream(dev)
     ab.ab_forward_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, bufs, dev)  # warm-up
+    if barrier is not None:
+        barrier()
     torch.cuda.synchronize(dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
@@ -421,10 +426,10 @@ def run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, steps):
         ab.ab_forward_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, bufs, dev)
     t1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = t0.elapsed_time(t1) / steps
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
     nbytes = Qc.numel() * 2
-    return {"value": round(dense_flop(w) / (ms * 1e-3) / 1e12, 3), "unit": UNIT,
-            "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": round(ms, 3),
+    return {"value": round(whole_job_value(w, world, ms), 3), "unit": UNIT,
+            "h2d_bytes_per_step": world * 3 * nbytes, "d2h_bytes_per_step": world * nbytes, "ms_per_step": round(ms, 3),
             "api": "ab_forward_host (pinned host Q/K/V in, host O out)"}
 
 
