@@ -52,7 +52,7 @@ def lib():
         L.orc_kmeans.argtypes = [_f32p, _ci, _ci, _ci, _ci, _f64p, _i32p, _vp]
         L.orc_kmeans.restype = _ci
         L.orc_block_mass.argtypes = [_f64p, _i32p, _ci, _ci, _f64p, _ci, _ci, _ci, _ci, _f64p]
-        L.orc_select_head.argtypes = [_f32p, _f32p, _ci, _ci, _ci, _ci, _ci, _ci, _vp, _ci,
+        L.orc_select_head.argtypes = [_f32p, _f32p, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _vp, _ci,
                                       _f64p, _vp, _vp]
         L.orc_budget.argtypes = [_ci, _cd]
         L.orc_budget.restype = _ci
@@ -66,7 +66,7 @@ def lib():
         L.orc_topk_row.restype = _ci
         L.orc_ht_sums.argtypes = [_f32p, _f32p, _f32p, _ci, _ci, _ci, _i32p, _u32p, _ci, _cd,
                                   _f64p, _f64p]
-        L.orc_ht_attention_block.argtypes = [_f32p, _f32p, _f32p, _ci, _ci, _ci, _ci, _ci,
+        L.orc_ht_attention_block.argtypes = [_f32p, _f32p, _f32p, _ci, _ci, _ci, _ci, _ci, _ci,
                                              _i32p, _u32p, _ci, _f64p]
         _lib = L
     return _lib
@@ -93,12 +93,17 @@ def budget(Nkv: int, keep_ratio: float) -> int:
 
 
 def dense_rows(Q, K, V, row0=0, nrows=None):
-    """Dense softmax(QK^T/sqrt(d))V for rows [row0, row0+nrows) of one head."""
+    """Dense softmax(QK^T/sqrt(d))V for rows [row0, row0+nrows) of one head.
+
+    Q is [L, d]; K and V are [Lk, d] (Lk = L for self-attention)."""
     Q, K, V = _f32(Q), _f32(K), _f32(V)
     L, d = Q.shape
+    Lk = K.shape[0]
+    assert V.shape == K.shape and K.shape[1] == d
     nrows = L - row0 if nrows is None else nrows
+    assert 0 <= row0 and row0 + nrows <= L
     O = np.zeros((nrows, d), np.float64)
-    lib().orc_dense_rows(Q, K, V, L, d, row0, nrows, O)
+    lib().orc_dense_rows(Q, K, V, Lk, d, row0, nrows, O)
     return O
 
 
@@ -132,16 +137,21 @@ def block_mass(mu, counts, n_i, Ksum, L, kv_block):
 
 
 def select_head(Q, K, q_block, kv_block, C, iters, rows=None, want_centroids=False):
-    """IBCS for one (b, h): returns P [nrows, Nkv] (and mu, counts)."""
+    """IBCS for one (b, h): returns P [nrows, Nkv] (and mu, counts).
+
+    Q is [L, d] (query blocks), K is [Lk, d] (KV blocks; Lk = L for
+    self-attention)."""
     Q, K = _f32(Q), _f32(K)
     L, d = Q.shape
-    Nq, Nkv = -(-L // q_block), -(-L // kv_block)
+    Lk = K.shape[0]
+    assert K.shape[1] == d
+    Nq, Nkv = -(-L // q_block), -(-Lk // kv_block)
     rows_a = None if rows is None else np.ascontiguousarray(rows, np.int32)
     nrows = Nq if rows is None else len(rows_a)
     P = np.zeros((nrows, Nkv), np.float64)
     mu = np.zeros((nrows, C, d), np.float64) if want_centroids else None
     cnt = np.zeros((nrows, C), np.int32) if want_centroids else None
-    lib().orc_select_head(Q, K, L, d, q_block, kv_block, C, iters, _ptr(rows_a), nrows, P,
+    lib().orc_select_head(Q, K, L, Lk, d, q_block, kv_block, C, iters, _ptr(rows_a), nrows, P,
                           _ptr(mu), _ptr(cnt))
     return (P, mu, cnt) if want_centroids else P
 
@@ -232,8 +242,11 @@ def ht_sums(q, K, V, kv_block, idx, pi_q32, shift):
 
 
 def ht_attention_block(Q, K, V, q_block, kv_block, i, idx, pi_q32, count):
+    """Reweighted attention of query block i: Q [L, d], K and V [Lk, d]."""
     Q, K, V = _f32(Q), _f32(K), _f32(V)
     L, d = Q.shape
+    Lk = K.shape[0]
+    assert V.shape == K.shape and K.shape[1] == d
     n_i = min(q_block, L - i * q_block)
     idx = np.ascontiguousarray(idx[:count], np.int32)
     pq = np.ascontiguousarray(pi_q32[:count], np.uint32)
@@ -241,7 +254,7 @@ def ht_attention_block(Q, K, V, q_block, kv_block, i, idx, pi_q32, count):
         idx = np.zeros(1, np.int32)
         pq = np.zeros(1, np.uint32)
     O = np.zeros((n_i, d), np.float64)
-    lib().orc_ht_attention_block(Q, K, V, L, d, q_block, kv_block, i, idx, pq, int(count), O)
+    lib().orc_ht_attention_block(Q, K, V, L, Lk, d, q_block, kv_block, i, idx, pq, int(count), O)
     return O
 
 

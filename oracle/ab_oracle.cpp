@@ -95,8 +95,9 @@ void orc_philox4x32_10(const uint32_t* ctr, const uint32_t* key, uint32_t* out) 
 // "Cross-Attention Nasıl Çalışır?": softmax(Q K^T / sqrt(d)) V; self-attention
 // ("Self-Attention ile Karşılaştırma") takes Q, K, V from one sequence.  The
 // AB-Attention page's "3D tam dikkat" is bidirectional: no mask.
-// One (b, h) slice: Q, K, V are [L, d] fp32; rows [row0, row0 + nrows) of the
-// output go to O [nrows, d].
+// One (b, h) slice: K, V are [L, d] fp32 (L keys), Q holds at least
+// row0 + nrows query rows of d (a sequence of its own length under
+// cross-attention); rows [row0, row0 + nrows) of the output go to O [nrows, d].
 // ---------------------------------------------------------------------------
 void orc_dense_rows(const float* Q, const float* K, const float* V, int L, int d,
                     int row0, int nrows, double* O) {
@@ -235,24 +236,27 @@ void orc_block_mass(const double* mu, const int32_t* counts, int C, int n_i,
 // ---------------------------------------------------------------------------
 // IBCS for one (b, h) slice: summaries, then k-means and block mass for the
 // query blocks listed in `rows` (nrows of them; rows == null means all Nq).
-// Q, K [L, d].  P [nrows, Nkv]; mu [nrows, C, d] and counts [nrows, C] may
+// Q [L, d] (queries), K [Lk, d] (keys): Lk = L for self-attention; under
+// cross-attention (Cross-Attention page, "Cross-Attention Nasıl Çalışır?")
+// the keys come from another sequence, so the query blocks follow L and the
+// KV blocks Lk.  P [nrows, Nkv]; mu [nrows, C, d] and counts [nrows, C] may
 // be null.
 // ---------------------------------------------------------------------------
-void orc_select_head(const float* Q, const float* K, int L, int d, int q_block, int kv_block,
+void orc_select_head(const float* Q, const float* K, int L, int Lk, int d, int q_block, int kv_block,
                      int C, int iters, const int32_t* rows, int nrows, double* P, double* mu,
                      int32_t* counts) {
   const int Nq = ceil_div(L, q_block);
-  const int Nkv = ceil_div(L, kv_block);
+  const int Nkv = ceil_div(Lk, kv_block);
   if (!rows) nrows = Nq;
   std::vector<double> ksum((size_t)Nkv * d);
-  orc_ksum(K, L, d, kv_block, ksum.data());
+  orc_ksum(K, Lk, d, kv_block, ksum.data());
   std::vector<double> m((size_t)C * d);
   std::vector<int32_t> cnt(C);
   for (int r = 0; r < nrows; ++r) {
     const int i = rows ? rows[r] : r;
     const int n_i = block_len(i, q_block, L);
     orc_kmeans(Q + (size_t)i * q_block * d, n_i, d, C, iters, m.data(), cnt.data(), nullptr);
-    orc_block_mass(m.data(), cnt.data(), C, n_i, ksum.data(), Nkv, L, kv_block, d,
+    orc_block_mass(m.data(), cnt.data(), C, n_i, ksum.data(), Nkv, Lk, kv_block, d,
                    P + (size_t)r * Nkv);
     if (mu) std::memcpy(mu + (size_t)r * C * d, m.data(), sizeof(double) * C * d);
     if (counts) std::memcpy(counts + (size_t)r * C, cnt.data(), sizeof(int32_t) * C);
@@ -458,9 +462,10 @@ void orc_ht_sums(const float* q, const float* K, const float* V, int L, int d, i
 // largest weighted logit max_{j kept, k in j} (s_k + ln(1/pi_j)).  Reading: an
 // empty list (count = 0) gives O = 0.  All queries of the block share its
 // list (block-sparse attention, AB-Attention page, "Darboğazı" section).
-// Q, K, V [L, d]; O [n_i, d].
+// Q [L, d]; K, V [Lk, d] (Lk = L for self-attention, another sequence's
+// length under cross-attention); O [n_i, d].
 // ---------------------------------------------------------------------------
-void orc_ht_attention_block(const float* Q, const float* K, const float* V, int L, int d,
+void orc_ht_attention_block(const float* Q, const float* K, const float* V, int L, int Lk, int d,
                             int q_block, int kv_block, int i, const int32_t* idx,
                             const uint32_t* pi_q32, int count, double* O) {
   const int n_i = block_len(i, q_block, L);
@@ -478,7 +483,7 @@ void orc_ht_attention_block(const float* Q, const float* K, const float* V, int 
       const int j = idx[t];
       const double pij = pi_q32[t] == 0 ? 4294967296.0 : (double)pi_q32[t];
       const double bias = std::log(4294967296.0 / pij);
-      const int n = block_len(j, kv_block, L);
+      const int n = block_len(j, kv_block, Lk);
       for (int rr = 0; rr < n; ++rr) {
         const int k = j * kv_block + rr;
         double dot = 0.0;
@@ -487,7 +492,7 @@ void orc_ht_attention_block(const float* Q, const float* K, const float* V, int 
       }
     }
     double den = 0.0;
-    orc_ht_sums(q, K, V, L, d, kv_block, idx, pi_q32, count, m, num.data(), &den);
+    orc_ht_sums(q, K, V, Lk, d, kv_block, idx, pi_q32, count, m, num.data(), &den);
     for (int e = 0; e < d; ++e) o[e] = num[e] / den;
   }
 }
