@@ -40,12 +40,14 @@ class ab_params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("L", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("q_block", ctypes.c_int32), ("kv_block", ctypes.c_int32),
                 ("C", ctypes.c_int32), ("kmeans_iters", ctypes.c_int32),
-                ("keep_ratio", ctypes.c_float), ("seed", ctypes.c_uint64)]
+                ("keep_ratio", ctypes.c_float), ("L_kv", ctypes.c_int32), ("seed", ctypes.c_uint64)]
 
 
 @dataclass(frozen=True)
 class Params:
-    """Problem description (mirrors ``ab_params``)."""
+    """Problem description (mirrors ``ab_params``).  ``L`` is the number of
+    queries per (b, h); ``L_kv`` the number of keys and values (0: the same as
+    ``L``, i.e. self-attention)."""
 
     B: int
     H: int
@@ -57,6 +59,11 @@ class Params:
     kmeans_iters: int = 3
     keep_ratio: float = 0.1
     seed: int = 42
+    L_kv: int = 0
+
+    @property
+    def Lk(self) -> int:
+        return self.L_kv if self.L_kv > 0 else self.L
 
     @property
     def Nq(self) -> int:
@@ -64,17 +71,19 @@ class Params:
 
     @property
     def Nkv(self) -> int:
-        return -(-self.L // self.kv_block)
+        return -(-self.Lk // self.kv_block)
 
     def c(self) -> ab_params:
         return ab_params(self.B, self.H, self.L, self.d, self.q_block, self.kv_block, self.C,
-                         self.kmeans_iters, float(self.keep_ratio), int(self.seed) & (2**64 - 1))
+                         self.kmeans_iters, float(self.keep_ratio), int(self.L_kv),
+                         int(self.seed) & (2**64 - 1))
 
     @staticmethod
     def of(w, seed: int = 42, **kw) -> "Params":
         """From a ``synthetic.Workload``."""
         args = dict(B=w.B, H=w.H, L=w.L, d=w.d, q_block=w.q_block, kv_block=w.kv_block, C=w.C,
-                    kmeans_iters=w.kmeans_iters, keep_ratio=w.keep_ratio, seed=seed)
+                    kmeans_iters=w.kmeans_iters, keep_ratio=w.keep_ratio, seed=seed,
+                    L_kv=w.Lk if w.Lk != w.L else 0)
         args.update(kw)
         return Params(**args)
 
@@ -128,13 +137,19 @@ def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def _check_qkv(p: Params, *ts):
+def _check_bf16(t, shape):
     import torch
-    for t in ts:
-        if t.dtype != torch.bfloat16 or tuple(t.shape) != (p.B, p.H, p.L, p.d) or not t.is_contiguous():
-            raise ValueError(f"expected contiguous bf16 [{p.B},{p.H},{p.L},{p.d}], got {t.dtype} {tuple(t.shape)}")
-        if not t.is_cuda:
-            raise ValueError("expected a CUDA tensor")
+    if t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous():
+        raise ValueError(f"expected contiguous bf16 {list(shape)}, got {t.dtype} {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+
+
+def _check_qkv(p: Params, Q, *kv):
+    """Q (and O) are [B, H, L, d]; K and V are [B, H, Lk, d]."""
+    _check_bf16(Q, (p.B, p.H, p.L, p.d))
+    for t in kv:
+        _check_bf16(t, (p.B, p.H, p.Lk, p.d))
 
 
 def budget(p: Params) -> int:
@@ -229,13 +244,15 @@ def ab_sample_topk(p: Params, P):
 
 
 def ab_attention(p: Params, Q, K, V, idx, pi_q32, count, out=None):
-    """Packed 1/pi-weighted block-sparse attention; returns O [B,H,L,d] bf16."""
+    """Packed 1/pi-weighted block-sparse attention; Q [B,H,L,d], K and V
+    [B,H,Lk,d]; returns O [B,H,L,d] bf16."""
     import torch
     _check_qkv(p, Q, K, V)
     for t, shape in ((idx, (p.B, p.H, p.Nq, p.Nkv)), (pi_q32, (p.B, p.H, p.Nq, p.Nkv)), (count, (p.B, p.H, p.Nq))):
         if t.dtype not in (torch.int32, torch.uint32) or tuple(t.shape) != shape or not t.is_contiguous():
             raise ValueError(f"list tensor must be contiguous int32 {shape}")
     O = torch.empty_like(Q) if out is None else out
+    _check_bf16(O, (p.B, p.H, p.L, p.d))
     _check(lib().ab_attention(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(pi_q32),
                               _ptr(count), _ptr(O), _stream(Q.device)), "ab_attention")
     return O
@@ -246,6 +263,7 @@ def ab_attention_dense(p: Params, Q, K, V, out=None):
     import torch
     _check_qkv(p, Q, K, V)
     O = torch.empty_like(Q) if out is None else out
+    _check_bf16(O, (p.B, p.H, p.L, p.d))
     _check(lib().ab_attention_dense(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
                                     _stream(Q.device)), "ab_attention_dense")
     return O
@@ -275,7 +293,11 @@ def ab_forward(p: Params, Q, K, V, bufs: Buffers | None = None) -> Buffers:
 
 
 def ab_forward_host(p: Params, Qh, Kh, Vh, Oh, Qd, Kd, Vd, bufs: Buffers, device):
-    """Host bf16 [B,H,L,d] in (Qh, Kh, Vh) -> host out (Oh); Qd/Kd/Vd are device staging buffers."""
+    """Host bf16 Qh [B,H,L,d], Kh and Vh [B,H,Lk,d] -> host out Oh [B,H,L,d];
+    Qd/Kd/Vd are device staging buffers of the same shapes."""
+    for t, n in ((Qh, p.L), (Kh, p.Lk), (Vh, p.Lk), (Oh, p.L), (Qd, p.L), (Kd, p.Lk), (Vd, p.Lk)):
+        if tuple(t.shape) != (p.B, p.H, n, p.d) or not t.is_contiguous():
+            raise ValueError(f"expected contiguous [{p.B},{p.H},{n},{p.d}], got {tuple(t.shape)}")
     _check(lib().ab_forward_host(ctypes.byref(p.c()), _ptr(Qh), _ptr(Kh), _ptr(Vh), _ptr(Oh), _ptr(Qd),
                                  _ptr(Kd), _ptr(Vd), _ptr(bufs.P), _ptr(bufs.idx), _ptr(bufs.pi_q32),
                                  _ptr(bufs.count), _ptr(bufs.O), _ptr(bufs.ws), bufs.ws.numel(),

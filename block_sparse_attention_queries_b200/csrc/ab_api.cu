@@ -20,7 +20,7 @@ namespace {
 using namespace ab;
 
 struct Dims {
-  int B, H, L, d, q_block, kv_block, C, iters;
+  int B, H, L, Lk, d, q_block, kv_block, C, iters;  // L queries, Lk keys per (b, h)
   int BH, Nq, Nkv, Kb;
   float keep;
   uint64_t seed;
@@ -40,6 +40,7 @@ int budget_of(int Nkv, double keep) {
 ab_status check_params(const ab_params* p, bool need_method, Dims* out) {
   if (!p) return AB_ERR_INVALID_ARG;
   if (p->B < 1 || p->H < 1 || p->L < 1 || p->L > (1 << 24)) return AB_ERR_INVALID_ARG;
+  if (p->L_kv < 0 || p->L_kv > (1 << 24)) return AB_ERR_INVALID_ARG;
   if (int64_t(p->B) * p->H > (int64_t(1) << 20)) return AB_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return p->d > 0 ? AB_ERR_UNSUPPORTED : AB_ERR_INVALID_ARG;
   if (p->q_block != 64 && p->q_block != 128) return p->q_block > 0 ? AB_ERR_UNSUPPORTED : AB_ERR_INVALID_ARG;
@@ -52,12 +53,12 @@ ab_status check_params(const ab_params* p, bool need_method, Dims* out) {
     if (!(p->keep_ratio > 0.f) || !(p->keep_ratio <= 1.f)) return AB_ERR_INVALID_ARG;
   }
   Dims d{};
-  d.B = p->B; d.H = p->H; d.L = p->L; d.d = p->d; d.q_block = p->q_block;
+  d.B = p->B; d.H = p->H; d.L = p->L; d.Lk = p->L_kv > 0 ? p->L_kv : p->L; d.d = p->d; d.q_block = p->q_block;
   d.kv_block = need_method ? p->kv_block : 16;
   d.C = p->C; d.iters = p->kmeans_iters; d.keep = p->keep_ratio; d.seed = p->seed;
   d.BH = p->B * p->H;
   d.Nq = (p->L + d.q_block - 1) / d.q_block;
-  d.Nkv = (p->L + d.kv_block - 1) / d.kv_block;
+  d.Nkv = (d.Lk + d.kv_block - 1) / d.kv_block;
   d.Kb = need_method ? budget_of(d.Nkv, double(p->keep_ratio)) : 0;
   if (int64_t(d.BH) * d.Nq > 0x7fffffff || int64_t(d.BH) * d.Nq * d.Nkv > (int64_t(1) << 40))
     return AB_ERR_INVALID_ARG;
@@ -149,7 +150,7 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, floa
   {
     const int64_t warps = int64_t(d.BH) * d.Nkv;
     ksum_kernel<D><<<unsigned((warps + 7) / 8), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(K), ksum,
-                                                              d.BH, d.L, d.Nkv, d.kv_block);
+                                                              d.BH, d.Lk, d.Nkv, d.kv_block);
     if (launch_status() != AB_OK) return AB_ERR_CUDA;
   }
   // k-means per query block
@@ -183,7 +184,7 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, floa
     a.counts_ws = cnt_ws;
     a.P = P;
     a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
-    const int n_last = d.L - (d.Nkv - 1) * d.kv_block;
+    const int n_last = d.Lk - (d.Nkv - 1) * d.kv_block;
     a.last_bias = float(std::log2(double(n_last) / double(d.kv_block)));
     const int G = 128 / d.C;
     const unsigned grid = unsigned(d.BH * ((d.Nq + G - 1) / G));
@@ -207,18 +208,18 @@ template <int D>
 ab_status run_attention(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* idx,
                         const uint32_t* pi_q32, const int32_t* count, void* O, bool dense, cudaStream_t st) {
   const int kvb = dense ? 128 : d.kv_block;
-  const bool grouped = (d.L % 8) == 0;
+  const bool grouped = (d.Lk % 8) == 0;
   CUtensorMap tmQ, tmK, tmV;
   if (!make_map(&tmQ, Q, D, d.L, d.BH, 128)) return AB_ERR_CUDA;
   if (grouped) {
-    if (!make_map_grouped(&tmK, K, D, d.L, d.BH, uint32_t(kvb / 8))) return AB_ERR_CUDA;
-    if (!make_map_grouped(&tmV, V, D, d.L, d.BH, uint32_t(kvb / 8))) return AB_ERR_CUDA;
+    if (!make_map_grouped(&tmK, K, D, d.Lk, d.BH, uint32_t(kvb / 8))) return AB_ERR_CUDA;
+    if (!make_map_grouped(&tmV, V, D, d.Lk, d.BH, uint32_t(kvb / 8))) return AB_ERR_CUDA;
   } else {
-    if (!make_map(&tmK, K, D, d.L, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
-    if (!make_map(&tmV, V, D, d.L, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
+    if (!make_map(&tmK, K, D, d.Lk, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
+    if (!make_map(&tmV, V, D, d.Lk, d.BH, uint32_t(kvb))) return AB_ERR_CUDA;
   }
   AttnArgs a{};
-  a.BH = d.BH; a.H = d.H; a.L = d.L; a.Nq = d.Nq; a.Nkv = dense ? (d.L + 127) / 128 : d.Nkv;
+  a.BH = d.BH; a.H = d.H; a.L = d.L; a.Lk = d.Lk; a.Nq = d.Nq; a.Nkv = dense ? (d.Lk + 127) / 128 : d.Nkv;
   a.q_block = d.q_block;
   a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
   a.O = reinterpret_cast<__nv_bfloat16*>(O);
@@ -455,20 +456,20 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
     return AB_ERR_INVALID_ARG;
   if (ws_bytes < workspace_layout(d).total) return AB_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t head_bytes = size_t(d.L) * d.d * 2;
+  const size_t q_head = size_t(d.L) * d.d * 2, kv_head = size_t(d.Lk) * d.d * 2;  // bytes per (b, h)
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return AB_ERR_CUDA;
   // groups of up to ceil(BH / 10) heads, a multiple of 4 so that every group's
   // row offset keeps the per-row buffers 16-byte aligned
   const int per = (((d.BH + 9) / 10) + 3) / 4 * 4;
   if (cap != cudaStreamCaptureStatusNone || per >= d.BH) {  // one stream: copies, path, copy back
-    const size_t bytes = size_t(d.BH) * head_bytes;
-    if (cudaMemcpyAsync(Q, Q_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
-    if (cudaMemcpyAsync(K, K_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
-    if (cudaMemcpyAsync(V, V_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
+    const size_t qb = size_t(d.BH) * q_head, kvb = size_t(d.BH) * kv_head;
+    if (cudaMemcpyAsync(Q, Q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
+    if (cudaMemcpyAsync(K, K_host, kvb, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
+    if (cudaMemcpyAsync(V, V_host, kvb, cudaMemcpyHostToDevice, st) != cudaSuccess) return AB_ERR_CUDA;
     s = ab_forward(p, Q, K, V, P, idx, pi_q32, count, O, workspace, ws_bytes, stream);
     if (s != AB_OK) return s;
-    if (cudaMemcpyAsync(O_host, O, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return AB_ERR_CUDA;
+    if (cudaMemcpyAsync(O_host, O, qb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return AB_ERR_CUDA;
     return AB_OK;
   }
   // Pipelined over groups of heads (every (b, h) is independent): the inputs
@@ -486,12 +487,13 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
   auto bw = [](void* base, size_t off) { return static_cast<uint8_t*>(base) + off; };
   for (int bh0 = 0; bh0 < d.BH; bh0 += per) {
     const int nbh = per < d.BH - bh0 ? per : d.BH - bh0;
-    const size_t off = size_t(bh0) * head_bytes, bytes = size_t(nbh) * head_bytes;
+    const size_t off = size_t(bh0) * q_head, bytes = size_t(nbh) * q_head;           // Q, O
+    const size_t koff = size_t(bh0) * kv_head, kbytes = size_t(nbh) * kv_head;       // K, V
     cudaEvent_t in_done, comp_done;
     if (!pipe.event(&in_done) || !pipe.event(&comp_done)) return AB_ERR_CUDA;
     if (cudaMemcpyAsync(bw(Q, off), bf(Q_host, off), bytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess ||
-        cudaMemcpyAsync(bw(K, off), bf(K_host, off), bytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess ||
-        cudaMemcpyAsync(bw(V, off), bf(V_host, off), bytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess)
+        cudaMemcpyAsync(bw(K, koff), bf(K_host, koff), kbytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess ||
+        cudaMemcpyAsync(bw(V, koff), bf(V_host, koff), kbytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess)
       return AB_ERR_CUDA;
     if (cudaEventRecord(in_done, pipe.in) != cudaSuccess) return AB_ERR_CUDA;
     if (cudaStreamWaitEvent(st, in_done, 0) != cudaSuccess) return AB_ERR_CUDA;
@@ -504,11 +506,11 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
     int32_t* idxc = idx + rows0 * d.Nkv;
     uint32_t* pic = pi_q32 + rows0 * d.Nkv;
     int32_t* cntc = count + rows0;
-    s = do_select(dc, bf(Q, off), bf(K, off), Pc, nullptr, nullptr, workspace, ws_bytes, st);
+    s = do_select(dc, bf(Q, off), bf(K, koff), Pc, nullptr, nullptr, workspace, ws_bytes, st);
     if (s != AB_OK) return s;
     s = do_sample(dc, Pc, idxc, pic, cntc, st, d.H, int64_t(rows0));
     if (s != AB_OK) return s;
-    s = do_attention(dc, bf(Q, off), bf(K, off), bf(V, off), idxc, pic, cntc, bw(O, off), false, st);
+    s = do_attention(dc, bf(Q, off), bf(K, koff), bf(V, koff), idxc, pic, cntc, bw(O, off), false, st);
     if (s != AB_OK) return s;
     if (cudaEventRecord(comp_done, st) != cudaSuccess) return AB_ERR_CUDA;
     if (cudaStreamWaitEvent(pipe.out, comp_done, 0) != cudaSuccess) return AB_ERR_CUDA;

@@ -50,7 +50,7 @@
 namespace ab {
 
 struct AttnArgs {
-  int BH, H, L, Nq, Nkv;
+  int BH, H, L, Lk, Nq, Nkv;  // L queries, Lk keys per (b, h)
   int q_block;  // 64 or 128
   const int32_t* idx;
   const uint32_t* pi_q32;
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (qi >= a.Nq) {
       cnt[s] = 0;
     } else if (kDense) {
-      cnt[s] = (a.L + 127) / 128;
+      cnt[s] = (a.Lk + 127) / 128;
     } else {
       int c = a.count[int64_t(bh) * a.Nq + qi];
       if (c < 0 || c > a.Nkv) {
@@ -273,10 +273,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (lane < kSlots) {
         if (kDense) {
           row = t * 128;
-          valid = min(128, a.L - row);
+          valid = min(128, a.Lk - row);
         } else if (j_cur >= 0) {
           row = j_cur * KVB;
-          valid = min(KVB, a.L - row);
+          valid = min(KVB, a.Lk - row);
           bias = pq_cur == 0u ? 0.f : 32.f - log2f(float(pq_cur));  // log2(1/pi), Pi = pq or 2^32
         }
       }
@@ -409,7 +409,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tO = tmem + 256u + uint32_t(s * D) + lane_base;
     const int qi = qi0 + s;
     float m_use = -INFINITY;  // reference max (log2 domain)
-    float l = 0.f;            // running sum of exp2(x - m_use)
+    // Running sum of the weights exp2(x - m_use) as the P V product sees them,
+    // i.e. rounded to bfloat16: O / l is then a weighted mean whose weights
+    // are exactly the bf16 P.  (With the lazy reference max the largest weight
+    // of a row is not 1 and its rounding would otherwise bias O toward 0.)
+    float l = 0.f;
     bool ok = true;
     // Keys [64h, 64h + 64) of P are stored: let the MMA warp use them.
     auto publish = [&](int h) {
@@ -457,7 +461,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       mbar_arrive(bar(kBarKEmpty + ks));
       tmem_wait_ld();
-      float lsum = 0.f;
+      float l_lo = 0.f, l_hi = 0.f;  // this tile's sum of the bf16 weights (even, odd columns)
       bool need;
       float alpha = 1.f;
       if (full) {
@@ -481,7 +485,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         rescale_O(need, alpha);
         const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
-        uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
@@ -497,15 +500,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               p0 = ex2_approx(p0);
               p1 = ex2_approx(p1);
             }
-            acc2 = f2_add(acc2, f2_pack(p0, p1));
             pk[k] = pack_bf16x2(p0, p1);
+            add_bf16x2_f32(pk[k], l_lo, l_hi);
           }
           tmem_st32_ptr(tS + uint32_t(32 * h), pk);
           publish(h);
         }
-        float s0, s1;
-        f2_unpack(acc2, s0, s1);
-        lsum = s0 + s1;
       } else {
         float rmax = -INFINITY;
 #pragma unroll
@@ -530,14 +530,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int k = 0; k < 32; ++k) {
             const float p0 = ex2_approx(x[64 * h + 2 * k] - mref);
             const float p1 = ex2_approx(x[64 * h + 2 * k + 1] - mref);
-            lsum += p0 + p1;
             pk[k] = pack_bf16x2(p0, p1);
+            add_bf16x2_f32(pk[k], l_lo, l_hi);
           }
           tmem_st32_ptr(tS + uint32_t(32 * h), pk);
           publish(h);
         }
       }
-      l += lsum;
+      l += l_lo + l_hi;
     }
     // ---------------------------------------------------------- epilogue
     if (qi < a.Nq) {

@@ -28,11 +28,15 @@
  *
  * Conventions shared by every call
  * --------------------------------
- *  - Tensors Q, K, V, O are [B, H, L, d] bfloat16, contiguous, d fastest,
- *    tokens in raster order of the (t, y, x) grid.  Query blocks are the
- *    contiguous runs of q_block tokens (Nq = ceil(L / q_block)); KV blocks
- *    the runs of kv_block tokens (Nkv = ceil(L / kv_block)); the last block of
- *    each kind may be partial.
+ *  - Tensors Q and O are [B, H, L, d], K and V are [B, H, Lk, d], all
+ *    bfloat16, contiguous, d fastest, tokens in raster order of the (t, y, x)
+ *    grid.  Lk = ab_params.L_kv, or L when L_kv is 0 (self-attention); under
+ *    cross-attention the keys and values come from a sequence of their own
+ *    length (Cross-Attention glossary page, "Cross-Attention Nasıl
+ *    Çalışır?").  Query blocks are the contiguous runs of q_block queries
+ *    (Nq = ceil(L / q_block)); KV blocks the runs of kv_block keys
+ *    (Nkv = ceil(Lk / kv_block)); the last block of each kind may be
+ *    partial.
  *  - Memory: the caller allocates and owns every buffer (device memory unless a
  *    call says "host"); the library allocates and frees no memory (only a
  *    pipelined ab_forward_host call creates, and releases, two streams and
@@ -76,12 +80,13 @@ typedef enum {
 
 /* Problem description shared by every call. */
 typedef struct {
-  int32_t B, H, L, d;        /* batch, heads, tokens, head dim; d in {64, 128}; 1 <= L <= 2^24 */
+  int32_t B, H, L, d;        /* batch, heads, query tokens, head dim; d in {64, 128}; 1 <= L <= 2^24 */
   int32_t q_block;           /* query block size, 64 or 128 */
   int32_t kv_block;          /* KV block size, 16, 32 or 64 */
   int32_t C;                 /* clusters per query block: 1, 2, 4, 8 or 16 */
   int32_t kmeans_iters;      /* Lloyd iterations, 1..16 (3 in the workloads) */
   float keep_ratio;          /* target kept fraction of KV blocks, in (0, 1] */
+  int32_t L_kv;              /* key/value tokens Lk, 0 <= L_kv <= 2^24; 0 means Lk = L */
   uint64_t seed;             /* Philox key of the SIP draws */
 } ab_params;
 
@@ -108,7 +113,8 @@ ab_status ab_workspace_size(const ab_params* p, size_t* bytes);
  * The centroid-summary product runs on the tensor cores in bfloat16 with fp32
  * accumulation, so P matches an exact evaluation to a few 1e-3 relative.
  *
- *   Q, K       device, [B, H, L, d] bf16.
+ *   Q          device, [B, H, L, d] bf16.
+ *   K          device, [B, H, Lk, d] bf16.
  *   P          device, out, [B, H, Nq, Nkv] fp32; each row sums to 1.
  *   centroids  device, out, optional (NULL), [B, H, Nq, C, d] fp32.
  *   counts     device, out, optional (NULL), [B, H, Nq, C] int32.
@@ -178,15 +184,16 @@ ab_status ab_sample_topk(const ab_params* p, const float* P, int32_t* idx, uint3
  * item: KV blocks much smaller than a tile are packed into full tensor-core
  * tiles).  For query q of block i, with s_k = q . k / sqrt(d) and
  * w_j = 2^32 / Pi_j (1 when pi_q32 = 0):
- *   O_q = sum_{j in list(i)} w_j sum_{k in j, k < L} e^{s_k} v_k
- *       / sum_{j in list(i)} w_j sum_{k in j, k < L} e^{s_k};
+ *   O_q = sum_{j in list(i)} w_j sum_{k in j, k < Lk} e^{s_k} v_k
+ *       / sum_{j in list(i)} w_j sum_{k in j, k < Lk} e^{s_k};
  * a query block with count 0 gets O = 0.  The lists may come from ab_sample
  * (ab_sample_systematic, ab_sample_topk) or from any other source, in any
  * order; each entry must
  * satisfy 0 <= idx < Nkv and count <= Nkv (violations raise AB_ERR_CAPACITY on
  * the device and the offending entries or rows are skipped).
  *
- *   Q, K, V  device, [B, H, L, d] bf16.
+ *   Q        device, [B, H, L, d] bf16.
+ *   K, V     device, [B, H, Lk, d] bf16.
  *   idx, pi_q32, count  device, as written by ab_sample.
  *   O        device, out, [B, H, L, d] bf16 (round to nearest even).
  */
@@ -196,8 +203,9 @@ ab_status ab_attention(const ab_params* p, const void* Q, const void* K, const v
 /*
  * Dense attention O = softmax(Q K^T / sqrt(d)) V, bidirectional, no mask
  * (Cross-Attention glossary page, "Cross-Attention Nasıl Çalışır?"; the
- * AB-Attention page's "3D tam dikkat").  Uses q_block (64 or 128), B, H, L, d
- * from *p; the other fields are ignored.  Same layout rules as ab_attention.
+ * AB-Attention page's "3D tam dikkat").  Uses q_block (64 or 128), B, H, L,
+ * L_kv, d from *p; the other fields are ignored.  Same layout rules as
+ * ab_attention.
  */
 ab_status ab_attention_dense(const ab_params* p, const void* Q, const void* K, const void* V, void* O,
                              void* stream);
@@ -212,10 +220,10 @@ ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const voi
                      size_t ws_bytes, void* stream);
 
 /*
- * ab_forward from HOST buffers: copies Q_host, K_host, V_host (host, [B, H, L,
- * d] bf16; page-locked memory gives asynchronous copies) to the device buffers
- * Q, K, V, runs the path, and copies O back to O_host (host, [B, H, L, d]
- * bf16).  Results are bit-identical to ab_forward on the same inputs.  When
+ * ab_forward from HOST buffers: copies Q_host (host, [B, H, L, d] bf16),
+ * K_host and V_host (host, [B, H, Lk, d] bf16; page-locked memory gives
+ * asynchronous copies) to the device buffers Q, K, V, runs the path, and
+ * copies O back to O_host (host, [B, H, L, d] bf16).  Results are bit-identical to ab_forward on the same inputs.  When
  * B * H > 4 and `stream` is not being captured, the call pipelines groups of
  * heads (every (b, h) is independent): the inputs of one group cross PCIe on
  * an internal stream while the previous group computes on `stream` and the

@@ -75,3 +75,38 @@ def test_status_strings(lib):
     for s in range(7):
         assert lib.ab_status_string(s)
     assert ab.status_string(6) == "workspace too small"
+
+
+def test_params_struct_matches_the_header(tmp_path):
+    """The ctypes mirror of ab_params has the C struct's size and offsets."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = [n for n, _ in ab.ab_params._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"ab.h\"\nint main(void) {\n"
+                   + "".join(f'  printf("%zu\\n", offsetof(ab_params, {n}));\n' for n in names)
+                   + '  printf("%zu\\n", sizeof(ab_params));\n  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.check_call([cc, "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    got = [int(x) for x in subprocess.check_output([str(exe)]).split()]
+    want = [getattr(ab.ab_params, n).offset for n in names] + [ctypes.sizeof(ab.ab_params)]
+    assert got == want
+
+
+def test_key_length_field(lib):
+    # cross-attention: Nkv follows L_kv, Nq follows L
+    p = ab.Params(B=1, H=3, L=8192, d=128, q_block=128, kv_block=16, C=8, keep_ratio=0.1, L_kv=3330)
+    assert (p.Nq, p.Nkv) == (64, 209)
+    assert ab.budget(p) == 21                      # floor(0.1 * 209 + 1/2)
+    assert ab.budget(ab.Params(B=1, H=3, L=8192, d=128, keep_ratio=0.1, L_kv=0)) == 51
+    ws = ab.workspace_size(p)
+    assert ws >= 3 * 209 * 128 * 2 + 3 * 64 * 8 * 128 * 2 + 3 * 64 * 8 * 4
+    assert ws < ab.workspace_size(ab.Params(B=1, H=3, L=8192, d=128, keep_ratio=0.1))
+    for bad in (-1, 2**24 + 1):
+        c = ab.Params(B=1, H=2, L=1000, d=128, L_kv=bad).c()
+        n = ctypes.c_size_t(0)
+        assert lib.ab_workspace_size(ctypes.byref(c), ctypes.byref(n)) == 1
+        assert lib.ab_budget(ctypes.byref(c)) == -1
