@@ -15,8 +15,8 @@ sample of (head, query block) rows against the oracle:
 
 Workloads: Wan2.1-480p (B=1, H=40, 21x30x52 tokens), HunyuanVideo-720p
 (H=24, 33x45x80 tokens; oracle on 2 heads x 16 query blocks) and the Wan-720p
-sweep (H=40, 21x45x80 tokens; KV block x keep ratio x C), plus dense
-attention at the Wan-720p shape.
+sweep (H=40, 21x45x80 tokens; KV block x keep ratio x C, and C = 1, the
+mean-query proxy), plus dense attention at the Wan-720p shape.
 """
 import numpy as np
 import pytest
@@ -137,6 +137,19 @@ def test_wan720_sweep(dev, kvb, keep, C):
     torch.cuda.synchronize()
     assert ab.device_error(dev) == 0
     _check_rows(p, host, bufs, heads=[0, w.H - 1], qblocks=_spread(p.Nq, 3), what=f"wan720 kvb{kvb} r{keep} C{C}")
+
+
+@pytest.mark.parametrize("kvb,keep", [(16, 0.10), (64, 0.05)])
+def test_wan720_mean_query_proxy(dev, kvb, keep):
+    # C = 1: one centroid per query block, the block's mean query, scores every
+    # KV block (a selector variant, the coarsest IBCS)
+    w = WORKLOADS["wan720"].with_(kv_block=kvb, keep_ratio=keep, C=1)
+    p = ab.Params.of(w)
+    host, (Q, K, V) = _workload_inputs("wan720", dev)
+    bufs = ab.ab_forward(p, Q, K, V)
+    torch.cuda.synchronize()
+    assert ab.device_error(dev) == 0
+    _check_rows(p, host, bufs, heads=[0, w.H - 1], qblocks=_spread(p.Nq, 3), what=f"wan720 C1 kvb{kvb} r{keep}")
 
 
 def test_wan720_dense_sampled_rows(dev):

@@ -11,11 +11,13 @@ Query blocks follow the query length L, KV blocks the key length Lk:
   too, with a ragged last query block and a ragged last KV block;
 * a subset of KV blocks attends to exactly those keys, never to keys beyond Lk;
 * IBCS closed forms with L != Lk: one cluster and one key per KV block gives
-  softmax_j(mean query . k_j / sqrt(d)); identical keys give P_j = n_j / Lk.
+  scipy's softmax_j(mean query . k_j / sqrt(d)); identical keys give
+  P_j = n_j / Lk.
 """
 import numpy as np
 import pytest
 import torch
+from scipy.special import softmax
 
 import oracle
 
@@ -23,11 +25,6 @@ import oracle
 def _sdpa64(q, K, V):
     t = lambda a: torch.from_numpy(np.asarray(a, np.float64))[None, None]
     return torch.nn.functional.scaled_dot_product_attention(t(q), t(K), t(V))[0, 0].numpy()
-
-
-def _softmax(x):
-    e = np.exp(x - x.max())
-    return e / e.sum()
 
 
 def _cross(L, Lk, d, seed):
@@ -80,7 +77,7 @@ def test_block_mass_cross_c1_bk1_is_softmax_of_mean_query():
     P = oracle.select_head(Q, K, q_block=64, kv_block=1, C=1, iters=3)
     assert P.shape == (1, Lk)
     qbar = Q.astype(np.float64).mean(0)
-    np.testing.assert_allclose(P[0], _softmax(K.astype(np.float64) @ qbar / np.sqrt(d)), rtol=1e-12)
+    np.testing.assert_allclose(P[0], softmax(K.astype(np.float64) @ qbar / np.sqrt(d)), rtol=1e-12)
 
 
 @pytest.mark.parametrize("L,Lk", [(100, 45), (30, 170)])
