@@ -11,7 +11,9 @@ than the 126 MB L2, so no explicit L2 flush is needed between steps.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Prints one JSON line (rank 0).  The metric is dense-equivalent attention
-TFLOP/s (4 B H L^2 d flop per layer / time per layer).  `--impl reference`
+TFLOP/s (4 B H L^2 d flop per layer / time per layer; 4 B H L Lk d for the
+cross-attention workload, whose keys and values come from a sequence of Lk
+tokens).  `--impl reference`
 times the CPU oracle (the reference arm of this repository) on a bounded
 sample of the same workload on the host cores.
 """
@@ -34,7 +36,8 @@ METRIC = "dense-equivalent attention TFLOPS/s + tensor-pipe util; ms per attenti
 UNIT = "TFLOP/s"
 WORKLOAD_NAMES = {"wan480": "wan2.1-14b-480p-self-attention",
                   "hunyuan720": "hunyuanvideo-720p-self-attention",
-                  "wan720": "wan-720p-self-attention"}
+                  "wan720": "wan-720p-self-attention",
+                  "cross_wan480": "wan2.1-480p-clip-to-9-frame-reference-cross-attention"}
 
 
 def workload(args):
@@ -55,14 +58,21 @@ def workload(args):
 
 
 def dense_flop(w) -> float:
-    return 4.0 * w.B * w.H * float(w.L) ** 2 * w.d
+    """4 B H L Lk d: QK^T and PV of dense attention (Lk = L for self-attention)."""
+    return 4.0 * w.B * w.H * float(w.L) * float(w.Lk) * w.d
 
 
 def config_dict(w, extra=None):
-    c = {"workload": WORKLOAD_NAMES[w.name], "B": w.B, "H": w.H, "grid_txy": list(w.grid), "L": w.L, "d": w.d,
-         "q_block": w.q_block, "kv_block": w.kv_block, "C": w.C, "kmeans_iters": w.kmeans_iters,
-         "keep_ratio": w.keep_ratio, "sampler_seed": 42, "data_seed": 1234,
-         "l2": "inputs larger than L2 (Q, K, V 335 MB each); no flush"}
+    q_mb = w.B * w.H * w.L * w.d * 2 / 1e6
+    kv_mb = w.B * w.H * w.Lk * w.d * 2 / 1e6
+    c = {"workload": WORKLOAD_NAMES.get(w.name, w.name), "B": w.B, "H": w.H, "grid_txy": list(w.grid), "L": w.L,
+         "d": w.d, "q_block": w.q_block, "kv_block": w.kv_block, "C": w.C, "kmeans_iters": w.kmeans_iters,
+         "keep_ratio": w.keep_ratio, "sampler_seed": 42, "data_seed": 1234}
+    if w.grid_kv is not None:
+        c.update({"grid_kv_txy": list(w.grid_kv), "L_kv": w.Lk})
+    big = min(q_mb, kv_mb) > 126
+    c["l2"] = (f"inputs larger than L2 (Q {q_mb:.0f} MB, K and V {kv_mb:.0f} MB each); no flush" if big
+               else f"Q {q_mb:.0f} MB, K and V {kv_mb:.0f} MB each; no flush")
     if extra:
         c.update(extra)
     return c
@@ -251,6 +261,23 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def executed_flop(w, cnt, idx) -> float:
+    """Algorithmic flop of the sparse attention on given lists:
+    4 d sum_{b,h,i} n_i sum_{j in S_i} n_j (n_j < kv_block only for the last,
+    partial KV block)."""
+    cnt = np.asarray(cnt, np.int64)
+    n_i = np.array([min(w.q_block, w.L - i * w.q_block) for i in range(w.Nq)], np.int64)
+    flop = 4.0 * w.d * float((n_i[None, None, :] * cnt * w.kv_block).sum())
+    n_last = w.Lk - (w.Nkv - 1) * w.kv_block
+    if n_last < w.kv_block:
+        # rows whose list holds the last KV block (lists are ascending: it is the last entry)
+        pos = np.maximum(cnt - 1, 0)
+        last = np.take_along_axis(np.asarray(idx), pos[..., None], axis=-1)[..., 0]
+        has = (cnt > 0) & (last == w.Nkv - 1)
+        flop -= 4.0 * w.d * float((n_i[None, None, :] * has * (w.kv_block - n_last)).sum())
+    return flop
+
+
 def whole_job_value(w, world: int, ms_step: float) -> float:
     """Dense-equivalent TFLOP/s of the whole job: every rank processes one layer per step."""
     return dense_flop(w) * world / (ms_step * 1e-3) / 1e12
@@ -325,24 +352,8 @@ def run_ours(args):
     if code:
         raise SystemExit(f"device error in the timed region: {ab.status_string(code)}")
 
-    # executed algorithmic attention flop from the last step's lists: 4 d sum_i n_i sum_{j in S_i} n_j
-    cnt = bufs.count.cpu().numpy().astype(np.int64)
-    idx = bufs.idx.cpu().numpy()
-    n_last = w.L - (w.Nkv - 1) * w.kv_block
-    last_kept = sum(int((idx[0, h, i, :cnt[0, h, i]] == w.Nkv - 1).any())
-                    for h in range(w.H) for i in range(w.Nq) if cnt[0, h, i] > 0)
-    n_i = np.array([min(w.q_block, w.L - i * w.q_block) for i in range(w.Nq)], np.int64)
-    keys = cnt * w.kv_block
-    exec_flop = 4.0 * w.d * float((n_i[None, None, :] * keys).sum())
-    # correct the (at most one per row) partial last KV block
-    if last_kept:
-        part = np.zeros_like(cnt)
-        for h in range(w.H):
-            for i in range(w.Nq):
-                c = cnt[0, h, i]
-                if c and (idx[0, h, i, :c] == w.Nkv - 1).any():
-                    part[0, h, i] = w.kv_block - n_last
-        exec_flop -= 4.0 * w.d * float((n_i[None, None, :] * part).sum())
+    cnt = bufs.count.cpu().numpy()
+    exec_flop = executed_flop(w, cnt, bufs.idx.cpu().numpy())
     kept_frac = float(cnt.sum()) / (w.B * w.H * w.Nq * w.Nkv)
 
     total_ms = max_over_ranks(total_ms, world, dev)
@@ -414,7 +425,7 @@ def run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, steps, world=1, barrier=None):
     import torch
     Qh, Kh, Vh = (t.pin_memory() for t in (Qc, Kc, Vc))
     Oh = torch.empty_like(Qc).pin_memory()
-    Qd, Kd, Vd = (torch.empty_like(Qc, device=dev) for _ in range(3))
+    Qd, Kd, Vd = (torch.empty_like(t, device=dev) for t in (Qc, Kc, Vc))
     stream = torch.cuda.current_stream(dev)
     ab.ab_forward_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, bufs, dev)  # warm-up
     if barrier is not None:
@@ -427,9 +438,10 @@ def run_e2e(ab, p, w, Qc, Kc, Vc, bufs, dev, steps, world=1, barrier=None):
     t1.record(stream)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
-    nbytes = Qc.numel() * 2
+    h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh))
+    d2h = Oh.numel() * Oh.element_size()
     return {"value": round(whole_job_value(w, world, ms), 3), "unit": UNIT,
-            "h2d_bytes_per_step": world * 3 * nbytes, "d2h_bytes_per_step": world * nbytes, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": world * h2d, "d2h_bytes_per_step": world * d2h, "ms_per_step": round(ms, 3),
             "api": "ab_forward_host (pinned host Q/K/V in, host O out)"}
 
 
@@ -564,7 +576,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--heads", type=int, default=None,
                     help="run a smaller case of the same layer with this many heads (profiling only)")
-    ap.add_argument("--workload", choices=["wan480", "hunyuan720", "wan720"], default="wan480",
+    ap.add_argument("--workload", choices=["wan480", "hunyuan720", "wan720", "cross_wan480"], default="wan480",
                     help="layer shape (default: the Wan2.1-480p headline workload)")
     ap.add_argument("--kv-block", type=int, default=None, help="KV block size override (sweeps)")
     ap.add_argument("--keep", type=float, default=None, help="keep ratio override (sweeps)")

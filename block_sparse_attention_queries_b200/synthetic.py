@@ -89,9 +89,10 @@ class Workload:
 
 
 # Workloads: the tiny case the oracle runs in full, a small video, the
-# Wan2.1-480p / HunyuanVideo-720p / Wan-720p self-attention shapes, and two
+# Wan2.1-480p / HunyuanVideo-720p / Wan-720p self-attention shapes, and
 # cross-attention cases (a clip attending to a shorter / a longer clip, ragged
-# key counts: 3330 keys is not a multiple of 8).
+# key counts: 3330 keys is not a multiple of 8; the Wan2.1-480p clip attending
+# to a 9-frame reference clip).
 WORKLOADS = {
     "tiny": Workload("tiny", 1, 1, (4, 16, 16), 64, 8, 64, 16, 4, 0.10),
     "small": Workload("small", 1, 4, (8, 32, 32), 128, 16, 128, 16, 8, 0.10),
@@ -102,6 +103,9 @@ WORKLOADS = {
                             grid_kv=(3, 30, 37)),
     "cross_long": Workload("cross_long", 2, 2, (3, 20, 30), 64, 8, 64, 32, 4, 0.15,
                            grid_kv=(9, 24, 40)),
+    # the Wan2.1-480p clip attending to a 9-frame reference clip of the same frame size
+    "cross_wan480": Workload("cross_wan480", 1, 40, (21, 30, 52), 128, 16, 128, 16, 8, 0.11,
+                             grid_kv=(9, 30, 52)),
 }
 
 

@@ -1,0 +1,47 @@
+"""Host-side arithmetic of bench.py on CPU: the executed attention flop of a
+set of lists (against a direct count over every kept block), the dense
+flop of self- and cross-attention, and the config record."""
+import os
+import sys
+
+import numpy as np
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+from block_sparse_attention_queries_b200.synthetic import WORKLOADS  # noqa: E402
+
+
+def _direct(w, cnt, idx):
+    tot = 0
+    for b in range(w.B):
+        for h in range(w.H):
+            for i in range(w.Nq):
+                n_i = min(w.q_block, w.L - i * w.q_block)
+                for j in idx[b, h, i, :cnt[b, h, i]]:
+                    tot += 4 * w.d * n_i * min(w.kv_block, w.Lk - int(j) * w.kv_block)
+    return float(tot)
+
+
+def test_executed_flop_matches_direct_count():
+    rng = np.random.default_rng(3)
+    for name in ("cross_short", "cross_long", "tiny"):
+        w = WORKLOADS[name]
+        cnt = rng.integers(0, w.Nkv + 1, size=(w.B, w.H, w.Nq)).astype(np.int32)
+        cnt[0, 0, 0] = w.Nkv          # a row holding the partial last block
+        cnt[-1, -1, -1] = 0           # an empty row
+        idx = np.zeros((w.B, w.H, w.Nq, w.Nkv), np.int32)
+        for r in np.ndindex(*cnt.shape):
+            idx[r][:cnt[r]] = np.sort(rng.choice(w.Nkv, cnt[r], replace=False))
+        assert bench.executed_flop(w, cnt, idx) == _direct(w, cnt, idx), name
+
+
+def test_dense_flop_and_config_of_cross_attention():
+    w = WORKLOADS["cross_wan480"]
+    assert (w.L, w.Lk) == (32760, 14040)
+    assert bench.dense_flop(w) == 4.0 * 40 * 32760 * 14040 * 128
+    s = WORKLOADS["wan480"]
+    assert bench.dense_flop(s) == 4.0 * 40 * 32760 ** 2 * 128
+    c = bench.config_dict(w)
+    assert c["L_kv"] == 14040 and c["grid_kv_txy"] == [9, 30, 52]
+    assert "L_kv" not in bench.config_dict(s)
+    assert c["l2"].startswith("inputs larger than L2")

@@ -16,7 +16,8 @@ sample of (head, query block) rows against the oracle:
 Workloads: Wan2.1-480p (B=1, H=40, 21x30x52 tokens), HunyuanVideo-720p
 (H=24, 33x45x80 tokens; oracle on 2 heads x 16 query blocks) and the Wan-720p
 sweep (H=40, 21x45x80 tokens; KV block x keep ratio x C, and C = 1, the
-mean-query proxy), plus dense attention at the Wan-720p shape.
+mean-query proxy), dense attention at the Wan-720p shape, and cross-attention
+of the Wan2.1-480p clip to a 9-frame reference clip (14040 keys).
 """
 import numpy as np
 import pytest
@@ -124,6 +125,19 @@ def test_hunyuan720_two_heads_sixteen_blocks(dev):
     torch.cuda.synchronize()
     assert ab.device_error(dev) == 0
     _check_rows(p, host, bufs, heads=[0, w.H - 1], qblocks=_spread(p.Nq, 16), what="hunyuan720")
+
+
+def test_cross_wan480_full_layer(dev):
+    # cross-attention at full size: the Wan2.1-480p clip (32760 queries)
+    # attending to a 9-frame reference clip (14040 keys)
+    w = WORKLOADS["cross_wan480"]
+    p = ab.Params.of(w)
+    assert p.L_kv == 14040
+    host, (Q, K, V) = _workload_inputs("cross_wan480", dev)
+    bufs = ab.ab_forward(p, Q, K, V)
+    torch.cuda.synchronize()
+    assert ab.device_error(dev) == 0
+    _check_rows(p, host, bufs, heads=[0, 21, 39], qblocks=_spread(p.Nq, 4), what="cross_wan480")
 
 
 @pytest.mark.parametrize("kvb", [16, 32, 64])
