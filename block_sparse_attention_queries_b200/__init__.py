@@ -197,50 +197,44 @@ def ab_select_static(p: Params, Q, K, want_centroids=False):
     return (P, cent, cnt) if want_centroids else P
 
 
-def ab_sample(p: Params, P):
-    """SIP: returns idx [B,H,Nq,Nkv] int32, pi_q32 [B,H,Nq,Nkv] uint32 (as int32 storage), count [B,H,Nq]."""
+def _list_outputs(p: Params, P, out):
+    """Checks P and returns (idx, pi_q32, count): `out` if given (checked), else new zeroed tensors."""
     import torch
     if P.dtype != torch.float32 or tuple(P.shape) != (p.B, p.H, p.Nq, p.Nkv) or not P.is_contiguous():
         raise ValueError("P must be contiguous fp32 [B,H,Nq,Nkv]")
     dev = P.device
-    idx = torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev)
-    piq = torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev)
-    cnt = torch.zeros(p.B, p.H, p.Nq, dtype=torch.int32, device=dev)
-    _check(lib().ab_sample(ctypes.byref(p.c()), _ptr(P), _ptr(idx), _ptr(piq), _ptr(cnt), _stream(dev)),
-           "ab_sample")
+    if out is None:
+        return (torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev),
+                torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev),
+                torch.zeros(p.B, p.H, p.Nq, dtype=torch.int32, device=dev))
+    for t, shape in zip(out, ((p.B, p.H, p.Nq, p.Nkv), (p.B, p.H, p.Nq, p.Nkv), (p.B, p.H, p.Nq))):
+        if t.dtype not in (torch.int32, torch.uint32) or tuple(t.shape) != shape or not t.is_contiguous() \
+                or t.device != dev:
+            raise ValueError(f"list output must be contiguous int32 {shape} on {dev}")
+    return tuple(out)
+
+
+def _lists_call(fn_name, p: Params, P, out=None):
+    idx, piq, cnt = _list_outputs(p, P, out)
+    _check(getattr(lib(), fn_name)(ctypes.byref(p.c()), _ptr(P), _ptr(idx), _ptr(piq), _ptr(cnt),
+                                   _stream(P.device)), fn_name)
     return idx, piq, cnt
 
 
-def _lists_call(fn_name, p: Params, P):
-    import torch
-    if P.dtype != torch.float32 or tuple(P.shape) != (p.B, p.H, p.Nq, p.Nkv) or not P.is_contiguous():
-        raise ValueError("P must be contiguous fp32 [B,H,Nq,Nkv]")
-    dev = P.device
-    idx = torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev)
-    piq = torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev)
-    cnt = torch.zeros(p.B, p.H, p.Nq, dtype=torch.int32, device=dev)
-    _check(getattr(lib(), fn_name)(ctypes.byref(p.c()), _ptr(P), _ptr(idx), _ptr(piq), _ptr(cnt), _stream(dev)),
-           fn_name)
-    return idx, piq, cnt
+def ab_sample(p: Params, P, out=None):
+    """SIP: returns idx [B,H,Nq,Nkv] int32, pi_q32 [B,H,Nq,Nkv] uint32 (as int32 storage), count [B,H,Nq].
+    `out` = (idx, pi_q32, count) writes into caller-owned tensors instead."""
+    return _lists_call("ab_sample", p, P, out)
 
 
-def ab_sample_systematic(p: Params, P):
+def ab_sample_systematic(p: Params, P, out=None):
     """Systematic sampling with SIP's inclusion probabilities: same outputs as ab_sample."""
-    return _lists_call("ab_sample_systematic", p, P)
+    return _lists_call("ab_sample_systematic", p, P, out)
 
 
-def ab_sample_topk(p: Params, P):
+def ab_sample_topk(p: Params, P, out=None):
     """Truncation (top-Kb by P, ties to the lower block, pi = 1): same outputs as ab_sample."""
-    import torch
-    if P.dtype != torch.float32 or tuple(P.shape) != (p.B, p.H, p.Nq, p.Nkv) or not P.is_contiguous():
-        raise ValueError("P must be contiguous fp32 [B,H,Nq,Nkv]")
-    dev = P.device
-    idx = torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev)
-    piq = torch.zeros(p.B, p.H, p.Nq, p.Nkv, dtype=torch.int32, device=dev)
-    cnt = torch.zeros(p.B, p.H, p.Nq, dtype=torch.int32, device=dev)
-    _check(lib().ab_sample_topk(ctypes.byref(p.c()), _ptr(P), _ptr(idx), _ptr(piq), _ptr(cnt), _stream(dev)),
-           "ab_sample_topk")
-    return idx, piq, cnt
+    return _lists_call("ab_sample_topk", p, P, out)
 
 
 def ab_attention(p: Params, Q, K, V, idx, pi_q32, count, out=None):

@@ -110,3 +110,18 @@ def test_key_length_field(lib):
         n = ctypes.c_size_t(0)
         assert lib.ab_workspace_size(ctypes.byref(c), ctypes.byref(n)) == 1
         assert lib.ab_budget(ctypes.byref(c)) == -1
+
+
+def test_list_outputs_are_checked_before_any_call():
+    import torch
+    p = ab.Params(B=1, H=2, L=300, d=64, q_block=64, kv_block=16, C=4)
+    P = torch.zeros(1, 2, p.Nq, p.Nkv)
+    good = (torch.zeros(1, 2, p.Nq, p.Nkv, dtype=torch.int32), torch.zeros(1, 2, p.Nq, p.Nkv, dtype=torch.int32),
+            torch.zeros(1, 2, p.Nq, dtype=torch.int32))
+    assert ab._list_outputs(p, P, good)[0] is good[0]
+    with pytest.raises(ValueError):
+        ab._list_outputs(p, P, (good[0], good[1], torch.zeros(1, 2, p.Nq + 1, dtype=torch.int32)))
+    with pytest.raises(ValueError):
+        ab._list_outputs(p, P, (good[0].float(), good[1], good[2]))
+    with pytest.raises(ValueError):
+        ab._list_outputs(p, P.double(), good)

@@ -155,6 +155,25 @@ def _skewed_P(B, H, Nq, Nkv, seed):
     return (P / P.sum(-1, keepdims=True)).astype(np.float32)
 
 
+def test_samplers_write_into_caller_buffers(dev):
+    # out=(idx, pi_q32, count): the same lists as the allocating call, written in place
+    p = ab.Params(B=1, H=2, L=3000, d=64, q_block=64, kv_block=16, C=4, keep_ratio=0.2, seed=11)
+    P = torch.rand(p.B, p.H, p.Nq, p.Nkv, generator=torch.Generator().manual_seed(4)).to(dev)
+    P = (P / P.sum(-1, keepdim=True)).contiguous()
+    for fn in (ab.ab_sample, ab.ab_sample_systematic, ab.ab_sample_topk):
+        ref = fn(p, P)
+        out = (torch.full_like(ref[0], -7), torch.full_like(ref[1], -7), torch.full_like(ref[2], -7))
+        got = fn(p, P, out=out)
+        torch.cuda.synchronize()
+        assert all(g.data_ptr() == o.data_ptr() for g, o in zip(got, out))
+        assert torch.equal(got[2], ref[2])
+        for r in range(p.Nq):
+            c = int(ref[2][0, 0, r])
+            assert torch.equal(got[0][0, 0, r, :c], ref[0][0, 0, r, :c])
+            assert torch.equal(got[1][0, 0, r, :c], ref[1][0, 0, r, :c])
+    _no_device_error(dev)
+
+
 @pytest.mark.parametrize("B,H,L,kvb,keep,seed", [(2, 3, 1000, 16, 0.1, 42), (1, 2, 4096, 16, 0.5, 7),
                                                  (2, 1, 8192, 32, 0.05, 2**63 + 12345),
                                                  (1, 1, 2000, 64, 1.0, 3), (1, 2, 118800, 16, 0.08, 42),
