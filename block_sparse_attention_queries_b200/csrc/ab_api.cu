@@ -275,7 +275,7 @@ ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q3
   a.row0 = row0;
   const int rows = d.BH * d.Nq;
   if (d.Nkv <= 2048) {  // one warp per row, the row in registers
-    sip_warp_kernel<16><<<unsigned((rows + 7) / 8), 256, 0, st>>>(a, rows);
+    sip_warp_kernel<16, false><<<unsigned((rows + 7) / 8), 256, 0, st>>>(a, rows);
   } else if (d.Nkv <= kSipSmemCap) {
     const int smem = 16 * ((d.Nkv + 3) / 4);
     if (smem > 48 * 1024 &&
@@ -370,7 +370,10 @@ ab_status ab_sample_systematic(const ab_params* p, const float* P, int32_t* idx,
   a.H = d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
   a.seed_lo = uint32_t(d.seed); a.seed_hi = uint32_t(d.seed >> 32);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d.Nkv <= kSipSmemCap) {
+  const int rows = d.BH * d.Nq;
+  if (d.Nkv <= 2048) {  // one warp per row, the row in registers
+    sip_warp_kernel<16, true><<<unsigned((rows + 7) / 8), 256, 0, st>>>(a, rows);
+  } else if (d.Nkv <= kSipSmemCap) {
     const int smem = 16 * ((d.Nkv + 3) / 4);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(sip_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)

@@ -336,8 +336,11 @@ __global__ void __launch_bounds__(kSipThreads) sip_kernel(const SipArgs a) {
 // arithmetic as sip_kernel (results are identical integers), with the
 // quantised row in registers and warp shuffles instead of block barriers.
 // Lane l owns blocks j = 128 k + 4 l + q (k < KMAX, q < 4), i.e. the same 4
-// consecutive blocks per Philox call.
-template <int KMAX>
+// consecutive blocks per Philox call.  kSystematic: systematic sampling with
+// the same Pi (as systematic_pass: one offset U per row, block j kept iff a
+// point U + m 2^32 lies in [C_j, C_j + Pi_j), C_j the running sum of Pi in
+// ascending j, here a warp scan per 128-block chunk).
+template <int KMAX, bool kSystematic>
 __global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows) {
   static_assert(KMAX * 4 * 16777216ull < 4294967296ull, "per-lane partial sums must fit 32 bits");
   const int lane = threadIdx.x & 31;
@@ -395,7 +398,60 @@ __global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows
   const uint32_t R32 = uint32_t(R);
   int32_t* out_idx = a.idx + int64_t(row) * Nkv;
   uint32_t* out_pi = a.pi_q32 + int64_t(row) * Nkv;
+  const double inv_s32 = S ? 4294967296.0 / double(S) : 0.0;
   int base = 0;
+  if constexpr (kSystematic) {
+    const uint64_t U = philox4x32_10(make_uint4(0xFFFFFFFFu, uint32_t(i), uint32_t(h), uint32_t(b)), a.seed_lo,
+                                     a.seed_hi).x;
+    auto points_below = [&](uint64_t x) -> uint64_t { return x > U ? ((x - U - 1) >> 32) + 1 : 0; };
+    uint64_t base_c = 0;  // sum of Pi over the earlier chunks
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+      if (128 * k >= Nkv) break;  // warp-uniform
+      const int j0 = 128 * k + 4 * lane;
+      uint64_t pis[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        pis[q] = j0 + q >= Nkv ? 0ull
+                 : w[k][q] >= theta ? (1ull << 32)
+                                    : uint64_t(pi_free(uint64_t(R32) * w[k][q], S_hi, S_lo, inv_s32));
+      const uint64_t mine = (pis[0] + pis[1]) + (pis[2] + pis[3]);
+      uint64_t incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint64_t C = base_c + incl - mine;
+      uint32_t keep_mask = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint64_t next = C + pis[q];
+        if (j0 + q < Nkv && points_below(next) - points_below(C) == 1) keep_mask |= 1u << q;
+        C = next;
+      }
+      const int kept = __popc(keep_mask);
+      int kincl = kept;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, kincl, o);
+        if (lane >= o) kincl += y;
+      }
+      int pos = base + kincl - kept;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (keep_mask & (1u << q)) {
+          out_idx[pos] = j0 + q;
+          out_pi[pos] = uint32_t(pis[q] & 0xFFFFFFFFull);
+          ++pos;
+        }
+      }
+      base += __shfl_sync(0xffffffffu, kincl, 31);
+      base_c += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) a.count[row] = base;
+    return;
+  }
 #pragma unroll
   for (int k = 0; k < KMAX; ++k) {
     if (128 * k >= Nkv) break;  // warp-uniform
@@ -433,7 +489,6 @@ __global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows
   __syncwarp();  // out_idx written by the other lanes is read below
 
   // ---- inclusion probabilities of the kept entries (as in sip_kernel)
-  const double inv_s32 = S ? 4294967296.0 / double(S) : 0.0;
   for (int e = lane; e < base; e += 32) {
     const int j = out_idx[e];
     const uint32_t wj = quantise_w(__ldg(P + j));

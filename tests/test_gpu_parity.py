@@ -248,8 +248,8 @@ def test_truncated_attention_small_workload(dev):
 
 @pytest.mark.parametrize("B,H,L,kvb,keep,seed", [(2, 3, 1000, 16, 0.1, 42), (1, 2, 4096, 16, 0.5, 7),
                                                  (2, 1, 8192, 32, 0.05, 2**63 + 12345),
-                                                 (1, 1, 2000, 64, 1.0, 3), (1, 2, 118800, 16, 0.08, 42),
-                                                 (1, 1, 262400, 16, 0.02, 5)])
+                                                 (1, 1, 2000, 64, 1.0, 3), (1, 2, 32760, 16, 0.11, 9),
+                                                 (1, 2, 118800, 16, 0.08, 42), (1, 1, 262400, 16, 0.02, 5)])
 def test_sample_systematic_bit_exact(dev, B, H, L, kvb, keep, seed):
     p = ab.Params(B=B, H=H, L=L, d=128, q_block=128, kv_block=kvb, C=8, keep_ratio=keep, seed=seed)
     Nq = min(p.Nq, 12) if L > 100000 else p.Nq
