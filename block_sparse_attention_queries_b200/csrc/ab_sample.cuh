@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows
 // Truncation, the selection SIP is contrasted with (AB-Attention page,
 // section "Video Difüzyon Modellerinde Dikkat (Attention) Darboğazı": pruned
 // blocks drop out of the softmax; SIP item: SIP estimates dense attention
-// "instead of truncating it").  One CTA (256 threads) per row keeps the Kb
+// rather than truncating it).  One CTA (256 threads) per row keeps the Kb
 // blocks with the largest P, ties to the lower j, in ascending order, with
 // pi = 1 (pi_q32 = 0).  P >= 0, so the order of the values is the order of
 // their bit patterns as unsigned integers: a 4-pass, 8-bit radix select finds

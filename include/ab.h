@@ -167,8 +167,8 @@ ab_status ab_sample_systematic(const ab_params* p, const float* P, int32_t* idx,
 /*
  * Truncation, the selection SIP replaces (AB-Attention page, section "Video
  * Difüzyon Modellerinde Dikkat (Attention) Darboğazı": pruned blocks vanish
- * from the softmax; SIP item: SIP estimates dense attention "instead of
- * truncating it").  For every row of P, keep the Kb blocks with the largest
+ * from the softmax; SIP item: SIP estimates dense attention rather than
+ * truncating it).  For every row of P, keep the Kb blocks with the largest
  * P (Kb as for ab_sample; ties to the lower block index), in ascending order,
  * with weight 1 (pi_q32 = 0); count = Kb.  Same arguments, layout, ownership
  * and errors as ab_sample; P must be >= 0 (as ab_select writes it).  With

@@ -201,8 +201,8 @@ int orc_kmeans(const float* Qb, int n, int d, int C, int iters, double* mu,
 
 // ---------------------------------------------------------------------------
 // IBCS, step 3: block-mass estimate of one query block (AB-Attention page,
-// IBCS item: "estimates block importance"; SIP item: sampling is "in
-// proportion to the IBCS estimates").  Reading: a KV block's attention mass
+// IBCS item: an estimate of each block's importance; SIP item: sampling
+// proportional to that estimate).  Reading: a KV block's attention mass
 // for centroid c is approximated by n_j exp(mu_c . kbar_j / sqrt(d)), i.e.
 // score S_cj = mu_c . kbar_j / sqrt(d) + ln n_j, normalised over j with a
 // softmax; the query block's estimate mixes the per-centroid distributions by
@@ -279,7 +279,7 @@ int orc_budget(int Nkv, double keep_ratio) {
 // AB-Attention page, section "Video Difüzyon Modellerinde Dikkat (Attention)
 // Darboğazı" (pruned blocks drop out of the softmax entirely) and section
 // "AB-Attention ve Üç Temel Yeniliği", SIP item (SIP estimates dense attention
-// "instead of truncating it").  Readings: the same IBCS estimate P and the
+// rather than truncating it).  Readings: the same IBCS estimate P and the
 // same budget Kb; keep the Kb blocks with the largest P, ties to the lower j;
 // no reweighting (pi = 1, stored as pi_q32 = 0); kept j in ascending order.
 // Returns count = Kb.
@@ -306,7 +306,7 @@ int orc_topk_row(const float* P, int Nkv, int Kb, int32_t* idx, uint32_t* pi_q32
 // Readings, in order:
 //  1. quantise: W_j = max(1, floor(P_j * 2^24)) (P_j is the fp32 estimate);
 //  2. inclusion probabilities proportional to W with capping at 1, summing to
-//     Kb ("probability proportional to size"): the capped set A grows until
+//     Kb (probability proportional to size): the capped set A grows until
 //     it is stable; with R = Kb - |A| and S = sum of W over j not in A, every
 //     j not in A with R W_j >= S joins A.  Then Pi_j = 2^32 for j in A and
 //     Pi_j = max(1, floor(R W_j 2^32 / S)) otherwise (pi_j = Pi_j / 2^32);
