@@ -57,7 +57,7 @@ struct SipArgs {
   int64_t row0;  // global index of the first row (for the draws' counters): rows are (b, h, i) in order
 };
 
-__device__ __forceinline__ uint32_t quantise_w(float p) {
+__host__ __device__ __forceinline__ uint32_t quantise_w(float p) {
   const float s = floorf(p * 16777216.0f);
   return s < 1.0f ? 1u : uint32_t(s);  // p <= 1, so s <= 2^24
 }
@@ -65,7 +65,7 @@ __device__ __forceinline__ uint32_t quantise_w(float p) {
 // a S <= X 2^32 for a < 2^32 + 1, S = S_hi 2^32 + S_lo < 2^64, X < 2^64:
 // a S = (a S_hi) 2^32 + a S_lo, compared without 128-bit products.
 // `a` is passed as a_minus_1 (so that a = 2^32 fits) .
-__device__ __forceinline__ bool mul_le_shift32(uint32_t a_minus_1, uint32_t S_hi, uint32_t S_lo, uint64_t X) {
+__host__ __device__ __forceinline__ bool mul_le_shift32(uint32_t a_minus_1, uint32_t S_hi, uint32_t S_lo, uint64_t X) {
   const uint64_t t = uint64_t(a_minus_1) * S_lo + S_lo;  // a S_lo < 2^64
   const uint64_t h = uint64_t(a_minus_1) * S_hi + S_hi;  // a S_hi
   if (h > X) return false;
@@ -76,7 +76,7 @@ __device__ __forceinline__ bool mul_le_shift32(uint32_t a_minus_1, uint32_t S_hi
 // Pi = max(1, floor(X 2^32 / S)) < 2^32 for a free block (X = R W < S): a
 // double estimate (error below one unit), then the exact test a S <= X 2^32
 // moves it to the largest such a.
-__device__ __forceinline__ uint32_t pi_free(uint64_t X, uint32_t S_hi, uint32_t S_lo, double inv_s32) {
+__host__ __device__ __forceinline__ uint32_t pi_free(uint64_t X, uint32_t S_hi, uint32_t S_lo, double inv_s32) {
   uint64_t est = uint64_t(double(X) * inv_s32);
   if (est > 0xFFFFFFFFull) est = 0xFFFFFFFFull;
   while (est > 0 && !mul_le_shift32(uint32_t(est - 1), S_hi, S_lo, X)) --est;
