@@ -115,9 +115,9 @@ __device__ __forceinline__ bool lane0_wait(uint32_t bar, uint32_t parity, volati
 // Merged tile order of two streams with T0 and T1 tiles.
 struct Merge {
   int T0, T1, m, longer;
-  __device__ Merge(int a, int b) : T0(a), T1(b), m(min(a, b)), longer(a >= b ? 0 : 1) {}
-  __device__ int total() const { return T0 + T1; }
-  __device__ void tile(int g, int& s, int& t) const {
+  __host__ __device__ Merge(int a, int b) : T0(a), T1(b), m(a < b ? a : b), longer(a >= b ? 0 : 1) {}
+  __host__ __device__ int total() const { return T0 + T1; }
+  __host__ __device__ void tile(int g, int& s, int& t) const {
     if (g < 2 * m) {
       s = g & 1;
       t = g >> 1;
@@ -126,7 +126,7 @@ struct Merge {
       t = g - m;
     }
   }
-  __device__ int index(int s, int t) const { return t < m ? 2 * t + s : m + t; }
+  __host__ __device__ int index(int s, int t) const { return t < m ? 2 * t + s : m + t; }
 };
 
 // D: head dim (64 or 128).  KVB: keys per list slot (16, 32, 64), or 128 for
