@@ -278,6 +278,16 @@ def executed_flop(w, cnt, idx) -> float:
     return flop
 
 
+def tile_flop(w, cnt) -> float:
+    """Tensor-core work of the sparse attention as executed: every query block
+    runs ceil(count / (128 / kv_block)) tiles of 128 keys, each an S product
+    and a P V product of 128 x 128 x d (the padding of a list's last tile and
+    of a ragged last query block included): 4 * 128 * 128 * d flop per tile."""
+    slots = 128 // w.kv_block
+    tiles = (np.asarray(cnt, np.int64) + slots - 1) // slots
+    return 4.0 * 128 * 128 * w.d * float(tiles.sum())
+
+
 def whole_job_value(w, world: int, ms_step: float) -> float:
     """Dense-equivalent TFLOP/s of the whole job: every rank processes one layer per step."""
     return dense_flop(w) * world / (ms_step * 1e-3) / 1e12
@@ -354,6 +364,7 @@ def run_ours(args):
 
     cnt = bufs.count.cpu().numpy()
     exec_flop = executed_flop(w, cnt, bufs.idx.cpu().numpy())
+    tiles_flop = tile_flop(w, cnt)
     kept_frac = float(cnt.sum()) / (w.B * w.H * w.Nq * w.Nkv)
 
     total_ms = max_over_ranks(total_ms, world, dev)
@@ -383,6 +394,8 @@ def run_ours(args):
             "ms_select": round(statistics.mean(sel_ms), 4), "ms_sample": round(statistics.mean(smp_ms), 4),
             "ms_attention": round(att_avg, 4),
             "executed_tflops_attention": round(achieved, 2),
+            "tile_tflops_attention": round(tiles_flop / (att_avg * 1e-3) / 1e12, 2),
+            "tile_frac_of_peak": round(tiles_flop / (att_avg * 1e-3) / 1e12 / bf16_peak, 4),
             "kept_block_fraction": round(kept_frac, 5),
             "dense_kernel_ms": round(dense_ms, 3),
             "speedup_vs_own_dense_kernel": round(dense_ms / ms_step, 3),

@@ -45,3 +45,19 @@ def test_dense_flop_and_config_of_cross_attention():
     assert c["L_kv"] == 14040 and c["grid_kv_txy"] == [9, 30, 52]
     assert "L_kv" not in bench.config_dict(s)
     assert c["l2"].startswith("inputs larger than L2")
+
+
+def test_tile_flop_counts_full_tiles():
+    w = WORKLOADS["cross_short"]                      # kv_block 16: 8 blocks per 128-key tile
+    cnt = np.array([[[0, 1, 8, 9, 16, 17]]], np.int32)
+    tiles = 0 + 1 + 1 + 2 + 2 + 3
+    assert bench.tile_flop(w, cnt) == 4.0 * 128 * 128 * w.d * tiles
+    w64 = WORKLOADS["cross_short"].with_(kv_block=64)  # 2 blocks per tile
+    assert bench.tile_flop(w64, np.array([3, 4, 5])) == 4.0 * 128 * 128 * w64.d * (2 + 2 + 3)
+    # never below the algorithmic count of the same lists
+    rng = np.random.default_rng(5)
+    c = rng.integers(0, w.Nkv + 1, size=(w.B, w.H, w.Nq)).astype(np.int32)
+    idx = np.zeros((w.B, w.H, w.Nq, w.Nkv), np.int32)
+    for r in np.ndindex(*c.shape):
+        idx[r][:c[r]] = np.sort(rng.choice(w.Nkv, c[r], replace=False))
+    assert bench.tile_flop(w, c) >= bench.executed_flop(w, c, idx)
