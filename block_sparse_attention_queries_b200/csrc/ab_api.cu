@@ -209,8 +209,11 @@ ab_status run_attention(const Dims& d, const void* Q, const void* K, const void*
                         const uint32_t* pi_q32, const int32_t* count, void* O, bool dense, cudaStream_t st) {
   const int kvb = dense ? 128 : d.kv_block;
   const bool grouped = (d.Lk % 8) == 0;
-  CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmQ, tmK, tmV, tmO;
   if (!make_map(&tmQ, Q, D, d.L, d.BH, 128)) return AB_ERR_CUDA;
+  // output tiles are stored q_block rows at a time (a 128-row tile holds two
+  // query blocks when q_block is 64)
+  if (!make_map(&tmO, O, D, d.L, d.BH, uint32_t(d.q_block))) return AB_ERR_CUDA;
   if (grouped) {
     if (!make_map_grouped(&tmK, K, D, d.Lk, d.BH, uint32_t(kvb / 8))) return AB_ERR_CUDA;
     if (!make_map_grouped(&tmV, V, D, d.Lk, d.BH, uint32_t(kvb / 8))) return AB_ERR_CUDA;
@@ -233,7 +236,7 @@ ab_status run_attention(const Dims& d, const void* Q, const void* K, const void*
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return AB_ERR_CUDA;
     if (fa.numRegs < kRegsLaunch) return AB_ERR_UNSUPPORTED;
     // one CTA per pair of query blocks (2k, 2k+1) of a (b, h)
-    kern<<<unsigned(d.BH * ((d.Nq + 1) / 2)), kAttnThreads, smem, st>>>(tmQ, tmK, tmV, a);
+    kern<<<unsigned(d.BH * ((d.Nq + 1) / 2)), kAttnThreads, smem, st>>>(tmQ, tmK, tmV, tmO, a);
     return launch_status();
   };
   if (grouped) {

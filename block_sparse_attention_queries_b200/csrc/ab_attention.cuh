@@ -79,7 +79,7 @@ struct AttnSmem {
   static constexpr int kOffMeta = kOffV + kVStages * kTile;  // per K stage: 8 biases, 8 valid counts
   static constexpr int kMetaStride = 64;
   static constexpr int kOffBar = kOffMeta + kKStages * kMetaStride;
-  static constexpr int kNumBars = 21;
+  static constexpr int kNumBars = 23;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
@@ -97,6 +97,7 @@ enum : int {
   kBarOFinal = 16, // 2 (per stream)
   kBarDrain = 18,
   kBarPHalf = 19,  // 2 (per stream, 128 arrivals): keys [0, 64) of P are in TMEM
+  kBarOStaged = 21,  // 2 (per stream, one arrival per warp): the output tile is in shared memory
 };
 
 // Warp-uniform bounded wait: every lane of the calling warp gets the same answer.
@@ -140,7 +141,8 @@ struct Merge {
 template <int D, int KVB, bool kGrouped>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     ab_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                        const AttnArgs a) {
   using SM = AttnSmem<D>;
   constexpr bool kDense = (KVB == 128);
   constexpr int kSlots = 128 / KVB;
@@ -179,6 +181,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   const Merge mg(T[0], T[1]);
   const int G = mg.total();
+  // Dense attention with two query blocks: both streams read the same K and V
+  // tiles (keys [128t, 128t+128)), so each is loaded once, into K stage t % 3
+  // and V stage t % 2, for merged tiles 2t and 2t+1; otherwise every merged
+  // tile g has stages of its own (g % 3, g % 2).
+  const bool share = kDense && T[0] == T[1];
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -189,10 +196,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar(kBarPFull + s), 128);
       mbar_init(bar(kBarPHalf + s), 128);
       mbar_init(bar(kBarOFinal + s), 1);
+      mbar_init(bar(kBarOStaged + s), 4);
     }
     for (int k = 0; k < 3; ++k) {
       mbar_init(bar(kBarKFull + k), 1);
-      mbar_init(bar(kBarKEmpty + k), 128);
+      mbar_init(bar(kBarKEmpty + k), share ? 256 : 128);  // the softmax warps of every stream that reads it
     }
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
@@ -206,6 +214,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
   }
   tc_fence_before();
   __syncthreads();
@@ -223,7 +232,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // slots' weights and valid-key counts with the K tile.
     const bool is_k = warp == 8;
     constexpr uint32_t kTileBytes = uint32_t(SM::kTile);
-    int issued[3] = {0, 0, 0}, issued_q[2] = {0, 0};
+    int loads = 0;  // tiles loaded into this ring
     if (is_k && lane == 0) {
       for (int s = 0; s < 2; ++s) {
         if (T[s] == 0) continue;
@@ -231,7 +240,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int sl = 0; sl < SM::kSlabs; ++sl)
           tma_load_3d(sbase + SM::kOffQ + s * SM::kTile + sl * SM::kSlab, &tmQ, bar(kBarQ + s), sl * 64,
                       (qi0 + s) * a.q_block, bh);
-        issued_q[s] = 1;
       }
     }
     // List entries are fetched two tiles ahead of their use, so that the
@@ -268,6 +276,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       fetch(u + 2, j_far, pq_far);
       int s, t;
       mg.tile(u, s, t);
+      if (share && s == 1) continue;  // stream 1 reads the tile stream 0 loaded
       float bias = 0.f;
       int valid = 0, row = 0;  // an empty slot reads any in-range rows (finite data), fully masked
       if (lane < kSlots) {
@@ -280,26 +289,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           bias = pq_cur == 0u ? 0.f : 32.f - log2f(float(pq_cur));  // log2(1/pi), Pi = pq or 2^32
         }
       }
-      const int st = u % nstage, use = u / nstage;
+      const int si = share ? t : u;  // position in this ring's sequence of loads
+      const int st = si % nstage, use = si / nstage;
       const uint32_t full = full0 + 8u * uint32_t(st), empty = empty0 + 8u * uint32_t(st);
       if (!lane0_wait(empty, (use & 1) ^ 1, abort_flag)) { ok = false; break; }
-      if (is_k) {
-        float b_all[kSlots];
-        int v_all[kSlots];
-#pragma unroll
-        for (int e = 0; e < kSlots; ++e) {
-          b_all[e] = __shfl_sync(0xffffffffu, bias, e);
-          v_all[e] = __shfl_sync(0xffffffffu, valid, e);
-        }
-        if (lane == 0) {
-          float* mb = reinterpret_cast<float*>(smem + SM::kOffMeta + st * SM::kMetaStride);
-          int* mv = reinterpret_cast<int*>(smem + SM::kOffMeta + st * SM::kMetaStride + 32);
-#pragma unroll
-          for (int e = 0; e < kSlots; ++e) {
-            mb[e] = b_all[e];
-            mv[e] = v_all[e];
-          }
-        }
+      if (is_k && lane < kSlots) {
+        // this slot's weight and valid-key count, published with the K tile
+        reinterpret_cast<float*>(smem + SM::kOffMeta + st * SM::kMetaStride)[lane] = bias;
+        reinterpret_cast<int*>(smem + SM::kOffMeta + st * SM::kMetaStride + 32)[lane] = valid;
       }
       if (lane == 0) mbar_arrive_expect_tx(full, kTileBytes);
       __syncwarp();
@@ -312,7 +309,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tma_load_3d(dst + sl * SM::kSlab + lane * KVB * 128, tm, full, sl * 64, row, bh);
         }
       }
-      issued[st] += 1;
+      ++loads;
       j_cur = j_next;
       pq_cur = pq_next;
       j_next = j_far;
@@ -320,10 +317,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     if (!ok && lane == 0) {
       // let the copies already issued land before shared memory is released
-      for (int k = 0; k < nstage; ++k)
-        if (issued[k]) mbar_wait_drain(full0 + 8u * uint32_t(k), (issued[k] - 1) & 1);
-      for (int s = 0; s < 2; ++s)
-        if (issued_q[s]) mbar_wait_drain(bar(kBarQ + s), 0);
+      // (the last load into stage k is the largest i < loads with i % nstage == k)
+      for (int k = 0; k < nstage && k < loads; ++k) {
+        const int last = loads - 1 - ((loads - 1 - k) % nstage);
+        mbar_wait_drain(full0 + 8u * uint32_t(k), (last / nstage) & 1);
+      }
+      if (is_k)
+        for (int s = 0; s < 2; ++s)
+          if (T[s] > 0) mbar_wait_drain(bar(kBarQ + s), 0);
     }
   } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA
@@ -342,9 +343,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int s = 0; s < 2 && ok; ++s)
         if (T[s] > 0) ok = mbar_wait(bar(kBarQ + s), 0, abort_flag);
       auto issue_S = [&](int s, int t) -> bool {
-        const int g = mg.index(s, t);
-        const int ks = g % 3;
-        if (!mbar_wait(bar(kBarKFull + ks), (g / 3) & 1, abort_flag)) return false;
+        const int ki = share ? t : mg.index(s, t);
+        const int ks = ki % 3;
+        if (!mbar_wait(bar(kBarKFull + ks), (ki / 3) & 1, abort_flag)) return false;
         tc_fence_after();
         // K tile: next 64 columns at kHalfK, 8-row groups kSboK apart
         constexpr uint32_t kHalfK = kGrouped ? 1024u : uint32_t(SM::kSlab);
@@ -372,14 +373,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // P V in two halves of 64 keys: the first starts as soon as the
         // softmax warps have stored keys [0, 64) of P
         if (!mbar_wait(bar(kBarPHalf + s), t & 1, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(bar(kBarVFull + (g & 1)), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+        const int vi = share ? t : g;  // V tile's position in the V ring's loads
+        if (!mbar_wait(bar(kBarVFull + (vi & 1)), (vi >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tO = tmem + 256u + uint32_t(s * D);
         const uint32_t tP = tmem + uint32_t(s) * 128u;
         // V tile (MN-major): 16 keys per k-step, next 64 columns at kLboV, next 8 keys at kSboV
         constexpr uint32_t kStepV = kGrouped ? 16u * uint32_t(SM::kSlabs) * 128u : 2048u;
         SmemDesc vd = vdesc0;
-        vd.lo += uint32_t(g & 1) * uint32_t(SM::kTile >> 4);
+        vd.lo += uint32_t(vi & 1) * uint32_t(SM::kTile >> 4);
         mma_bf16_ts(tO, tP, desc_at(vd, 0), idO, t > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 1; kk < 4; ++kk) mma_bf16_ts(tO, tP + uint32_t(kk * 8), desc_at(vd, kk * kStepV), idO, 1u);
@@ -387,7 +389,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 4; kk < 8; ++kk) mma_bf16_ts(tO, tP + uint32_t(kk * 8), desc_at(vd, kk * kStepV), idO, 1u);
-        mma_commit(bar(kBarVEmpty + (g & 1)));
+        if (!share || s == 1) mma_commit(bar(kBarVEmpty + (vi & 1)));  // shared: after both streams' P V
         if (t + 1 < T[s]) {
           ok = issue_S(s, t + 1);
         } else {
@@ -439,10 +441,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       };
-      const int g = mg.index(s, t);
-      const int ks = g % 3;
+      const int ki = share ? t : mg.index(s, t);  // K tile's position in the K ring's loads
+      const int ks = ki % 3;
       if (!warp_wait(bar(kBarSFull + s), t & 1, abort_flag)) { ok = false; break; }
-      if (!warp_wait(bar(kBarKFull + ks), (g / 3) & 1, abort_flag)) { ok = false; break; }
+      if (!warp_wait(bar(kBarKFull + ks), (ki / 3) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float x[128];
 #pragma unroll
@@ -540,30 +542,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       l += l_lo + l_hi;
     }
     // ---------------------------------------------------------- epilogue
+    // O / l rounded to bf16 is staged in this stream's Q buffer (no MMA reads
+    // it any more once O is final) in the 128B-swizzled [half][row][128 B]
+    // layout, then written by TMA stores of {64 columns, q_block rows}: whole
+    // 128-byte lines, rows past the sequence clipped by the tensor map.  A
+    // stream without tiles writes zeros (O = 0 for an empty list).
     if (qi < a.Nq) {
-      const int n_i = min(a.q_block, a.L - qi * a.q_block);
-      __nv_bfloat16* orow = a.O + (int64_t(bh) * a.L + int64_t(qi) * a.q_block + r) * D;
       if (T[s] > 0 && ok) ok = warp_wait(bar(kBarOFinal + s), 0, abort_flag);
-      if (T[s] > 0 && ok) {
-        tc_fence_after();
-        const float inv = 1.f / l;
-        uint32_t o[D];
+      uint8_t* stage = smem + SM::kOffQ + s * SM::kTile;
+      if (ok) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;  // a row whose keys were all masked gets 0
+        if (T[s] > 0) tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32_nowait(tO + uint32_t(c * 32), o + c * 32);
-        tmem_wait_ld();
-        if (r < n_i) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          if (T[s] > 0) {
+            tmem_ld32(tO + uint32_t(c * 32), o);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int q = 0; q < D / 8; ++q) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + q * 8) = w;
+            for (int k = 0; k < 32; ++k) o[k] = 0u;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+            const int col = c * 32 + q * 8;  // first of the 8 columns
+            *reinterpret_cast<uint4*>(stage + (col / 64) * SM::kSlab + sw128_offset(uint32_t(r), uint32_t((col % 64) / 8))) = v;
           }
         }
-      } else if (T[s] == 0 && r < n_i) {
-        for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4*>(orow + c * 8) = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();  // the TMA store reads what the generic proxy wrote
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarOStaged + s));
+      if ((warp & 3) == 0 && lane == 0 && ok && mbar_wait(bar(kBarOStaged + s), 0, abort_flag)) {
+        for (int sl = 0; sl < SM::kSlabs; ++sl)
+          tma_store_3d(&tmO, smem_u32(stage) + uint32_t(sl * SM::kSlab), sl * 64, qi * a.q_block, bh);
+        bulk_commit_group();
+        bulk_wait_read_all();  // shared memory stays valid until the stores have read it
       }
     }
   }
