@@ -306,24 +306,52 @@ ab_status do_attention(const Dims& d, const void* Q, const void* K, const void* 
 // ------------------------------------------- scratch for ab_select_static
 // One file-scope device array serves every ab_select_static call on a device.
 // Host code cannot use the symbol itself as a device address; its address is
-// looked up once per device with cudaGetSymbolAddress.
+// looked up with cudaGetSymbolAddress, with the device current.  The address
+// belongs to the CUDA context it was looked up in, so it is cached per device
+// together with that context and looked up again when the calling thread's
+// current context is another one (a context made current by a host
+// framework, or a new primary context after a device reset).
 static __device__ __align__(256) uint8_t g_select_scratch[AB_SELECT_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+struct ScratchAddr {
+  CUcontext ctx;
+  void* ptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_select_scratch on the current device (nullptr on failure).
+PFN_cuCtxGetCurrent_v4000 ctx_current_fn() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &ptr, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+  });
+  return fn;
+}
+
+// Device address of g_select_scratch in the calling thread's current context
+// (nullptr on failure).
 void* static_scratch_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  auto get_ctx = ctx_current_fn();
+  if (!get_ctx) return nullptr;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;  // null before the thread's first runtime call
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess || !ptr) return nullptr;
-    g_scratch_addr[dev] = ptr;
-  }
-  return g_scratch_addr[dev];
+  ScratchAddr& e = g_scratch_addr[dev];
+  if (ctx && e.ptr && e.ctx == ctx) return e.ptr;
+  void* ptr = nullptr;  // the lookup also makes the device's context current if none was
+  if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess || !ptr) return nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
+  e.ctx = ctx;
+  e.ptr = ptr;
+  return ptr;
 }
 
 }  // namespace

@@ -59,7 +59,6 @@ struct AttnArgs {
   float scale_log2;  // log2(e) / sqrt(d)
 };
 
-constexpr int kPolyEvery = 0;  // > 0: one column pair in kPolyEvery takes exp2 on the FMA pipe (off: measured slower)
 constexpr int kAttnThreads = 384;
 constexpr int kRegsLaunch = 168;   // registers per thread the kernel is launched with
 constexpr int kRegsCtl = 56;       // producer / MMA warpgroup after re-balancing
@@ -496,12 +495,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float off = s_bias[c / KVB] - m_use;
             float p0, p1;
             f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), sc2, f2_pack(off, off)), p0, p1);
-            if (kPolyEvery > 0 && k % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
-              exp2_poly2(p0, p1);  // a share of the exponentials on the FMA pipe
-            } else {
-              p0 = ex2_approx(p0);
-              p1 = ex2_approx(p1);
-            }
+            p0 = ex2_approx(p0);
+            p1 = ex2_approx(p1);
             pk[k] = pack_bf16x2(p0, p1);
             add_bf16x2_f32(pk[k], l_lo, l_hi);
           }

@@ -347,37 +347,10 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// 2^a, 2^b on the FMA pipe (instead of MUFU) for a, b <= 64: Cody-Waite split
-// y = n + f, n = round(y) via the 1.5 * 2^23 rounding constant, f in [-1/2, 1/2];
-// 2^f from a cubic fitted for minimal relative error (7.5e-5, see
-// fit_exp2_poly.py); 2^n added to the exponent bits.  Inputs are clamped at
-// -125 so that the result stays a normal number (2^-125 stands in for smaller
-// values); callers use it only where no input is -inf.
-__device__ __forceinline__ void exp2_poly2(float& a, float& b) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t y = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
-  const uint64_t t = f2_add(y, f2_pack(kRound, kRound));
-  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), y);
-  uint64_t p = f2_fma(f, f2_pack(0.05517119169f, 0.05517119169f), f2_pack(0.2426111251f, 0.2426111251f));
-  p = f2_fma(p, f, f2_pack(0.6932610869f, 0.6932610869f));
-  p = f2_fma(p, f, f2_pack(0.9999280572f, 0.9999280572f));
-  float pa, pb, ta, tb;
-  f2_unpack(p, pa, pb);
-  f2_unpack(t, ta, tb);
-  a = __int_as_float(__float_as_int(pa) + ((__float_as_int(ta) - 0x4B400000) << 23));
-  b = __int_as_float(__float_as_int(pb) + ((__float_as_int(tb) - 0x4B400000) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -292,17 +292,21 @@ __global__ void __launch_bounds__(128, C <= 8 ? 5 : 3) kmeans_kernel(const __gri
     }
   }
 
-  if (ok) {
+  {
+    // A wait that gave up (AB_ERR_TIMEOUT recorded) leaves markers instead
+    // of results: NaN centroids and count -1, so that the scores built from
+    // them are NaN rather than values left in the workspace by an earlier call.
     const int64_t row0 = (int64_t(bh) * Nq + qi) * C;
 #pragma unroll
     for (int c = 0; c < C; ++c) {
       if (own_dim) {
-        if (cent_out) cent_out[(row0 + c) * D + tid] = mu[c];
-        cent_ws[(row0 + c) * D + tid] = __float2bfloat16_rn(mu[c]);
+        const float m = ok ? mu[c] : __uint_as_float(0x7fc00000u);
+        if (cent_out) cent_out[(row0 + c) * D + tid] = m;
+        cent_ws[(row0 + c) * D + tid] = __float2bfloat16_rn(m);
       }
       if (tid == c) {
-        if (counts_out) counts_out[row0 + c] = cnt[c];
-        counts_ws[row0 + c] = cnt[c];
+        if (counts_out) counts_out[row0 + c] = ok ? cnt[c] : -1;
+        counts_ws[row0 + c] = ok ? cnt[c] : -1;
       }
     }
   }

@@ -264,8 +264,13 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
  * that device current); make that first call before any stream capture.
  * Every call on a device shares the one array and leaves its contents behind;
  * nothing in it needs to start at zero, because each call writes every byte
- * it reads.  Calls whose work overlaps on the GPU (other streams, other host
- * threads) race on the array: order them on one stream or synchronise.
+ * it reads, the failure path included (a k-means wait that gives up writes
+ * NaN centroids and count -1, so that call's P is NaN and AB_ERR_TIMEOUT is
+ * in the device error word).  Calls whose work overlaps on the GPU (other
+ * streams, other host threads) race on the array: order them on one stream or
+ * synchronise.  The array's address belongs to a CUDA context: it is looked
+ * up again whenever the calling thread's current context differs from the one
+ * it was looked up in.
  */
 ab_status ab_select_static(const ab_params* p, const void* Q, const void* K, float* P, float* centroids,
                            int32_t* counts, void* stream);

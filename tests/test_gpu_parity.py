@@ -144,6 +144,18 @@ def test_bad_lists_raise_capacity_without_fault(dev):
     torch.cuda.synchronize()
     assert ab.device_error(dev) == 4  # AB_ERR_CAPACITY
     assert ab.device_error(dev) == 0  # cleared by the read
+    # a list whose every entry is invalid leaves no key: that block's output is
+    # 0 (as for an empty list), not NaN; the other block is unaffected
+    cnt2 = torch.tensor([[[2, 1]]], dtype=torch.int32, device=dev)
+    idx2 = torch.zeros_like(idx)
+    idx2[0, 0, 0, :2] = torch.tensor([16, -5])   # Nkv = 16: both out of range
+    idx2[0, 0, 1, 0] = 3
+    O = ab.ab_attention(p, Q, K, V, idx2, piq, cnt2)
+    torch.cuda.synchronize()
+    assert ab.device_error(dev) == 4
+    O0 = O[0, 0, :128].float()
+    assert torch.equal(O0, torch.zeros_like(O0))
+    assert torch.isfinite(O[0, 0, 128:].float()).all()
 
 
 # ------------------------------------------------------------------ sampler

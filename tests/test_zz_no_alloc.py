@@ -2,9 +2,9 @@
 fixed device array, for callers that cannot allocate device memory (plugins
 under a host framework's memory planner, code that must not block on
 cudaMalloc).  Checked through the C ABI against ab_select with a
-caller-supplied workspace, on two calls in a row (the array keeps the first
-call's contents, which the second must not depend on).  This file is
-collected last on purpose."""
+caller-supplied workspace, on two calls in a row that follow a call on a
+different problem (the array keeps each call's contents, which the next call
+must not depend on).  This file is collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -31,17 +31,30 @@ def _select_static(lib, p, Q, K, dev):
     return P, cent, cnt
 
 
-@pytest.mark.parametrize("wname", ["small", "tiny"])
-def test_select_static_matches_workspace_select(wname):
+def _dev():
     if not torch.cuda.is_available():
         pytest.fail("no CUDA device")
-    dev = torch.device("cuda:0")
-    lib = ab.lib()
+    return torch.device("cuda:0")
+
+
+def _case(wname, seed, dev):
     w = WORKLOADS[wname]
     p = ab.Params.of(w)
-    Qc, Kc, _ = make_workload_qkv(w)
-    Q, K = Qc.to(dev), Kc.to(dev)
+    Qc, Kc, _ = make_workload_qkv(w, seed=seed)
+    return p, Qc.to(dev), Kc.to(dev)
+
+
+@pytest.mark.parametrize("wname,other", [("small", "tiny"), ("tiny", "small")])
+def test_select_static_matches_workspace_select(wname, other):
+    # Each checked call follows a call on a different problem (other shape,
+    # other inputs), so what that call left in the shared array differs from
+    # what this one needs; then the check is repeated on a second call in a row.
+    dev = _dev()
+    lib = ab.lib()
+    p, Q, K = _case(wname, 1234, dev)
     P_ref, c_ref, n_ref = ab.ab_select(p, Q, K, want_centroids=True)
+    po, Qo, Ko = _case(other, 777, dev)
+    _select_static(lib, po, Qo, Ko, dev)
     for _ in range(2):
         P, cent, cnt = _select_static(lib, p, Q, K, dev)
         torch.cuda.synchronize()
@@ -53,11 +66,17 @@ def test_select_static_matches_workspace_select(wname):
 
 
 def test_select_static_rejects_problems_beyond_the_limit():
+    dev = _dev()
     lib = ab.lib()
-    # HunyuanVideo-720p layer: 91 MB of scratch > 48 MiB; rejected before any launch
+    # HunyuanVideo-720p layer: 91 MB of scratch > 48 MiB; rejected before any
+    # launch (the buffers are real, small device tensors: nothing reads them)
     w = WORKLOADS["hunyuan720"]
     p = ab.Params.of(w)
     assert ab.workspace_size(p) > 48 * 1024 * 1024
-    fake = ctypes.c_void_p(0x10000)
-    s = lib.ab_select_static(ctypes.byref(p.c()), fake, fake, fake, None, None, None)
+    buf = torch.zeros(1024, dtype=torch.float32, device=dev)
+    ptr = ctypes.c_void_p(buf.data_ptr())
+    st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    s = lib.ab_select_static(ctypes.byref(p.c()), ptr, ptr, ptr, None, None, st)
     assert s == AB_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert torch.equal(buf, torch.zeros_like(buf))
