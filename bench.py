@@ -9,6 +9,7 @@ outlier tokens) at the workload's shapes; each of Q, K, V is 335 MB, larger
 than the 126 MB L2, so no explicit L2 flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--split replicas|heads]
 
 Prints one JSON line (rank 0).  The metric is dense-equivalent attention
 TFLOP/s (4 B H L^2 d flop per layer / time per layer; 4 B H L Lk d for the
@@ -16,6 +17,12 @@ cross-attention workload, whose keys and values come from a sequence of Lk
 tokens).  `--impl reference`
 times the CPU oracle (the reference arm of this repository) on a bounded
 sample of the same workload on the host cores.
+
+Multi-GPU (one process per GPU): `--split replicas` (default) runs one whole
+layer per GPU (weak scaling); `--split heads` divides ONE layer's heads among
+the GPUs (ab_forward_slice on each GPU's contiguous slice, strong scaling).
+Either way no data crosses between GPUs: every (b, h) is independent on the
+path; NCCL carries only the barrier and the max-over-ranks time.
 """
 from __future__ import annotations
 
@@ -416,6 +423,96 @@ def run_ours(args):
     return out
 
 
+def run_ours_split(args):
+    """One layer per step, its heads divided among the ranks (ab_forward_slice
+    on every rank's contiguous slice of the B*H heads); the step time is the
+    slowest rank's and the value the layer's dense-equivalent rate."""
+    import torch
+    import torch.distributed as dist
+    import block_sparse_attention_queries_b200 as ab
+    from block_sparse_attention_queries_b200.synthetic import make_workload_qkv
+
+    rank, world, local = dist_env(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", rank=rank, world_size=world, device_id=dev,
+                                timeout=datetime.timedelta(seconds=120))
+    w = workload(args)
+    p = ab.Params.of(w, seed=42)
+    bh0, nbh = ab.head_slices(w.B, w.H, world)[rank]
+    Qc, Kc, Vc = make_workload_qkv(w)  # the whole layer, the same on every rank; each keeps its slice
+    Qs, Ks, Vs = (t.reshape(1, w.B * w.H, *t.shape[2:])[:, bh0:bh0 + nbh].contiguous() for t in (Qc, Kc, Vc))
+    Q, K, V = (t.to(dev) for t in (Qs, Ks, Vs))
+    bufs = ab.Buffers(ab.slice_params(p, nbh), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        ab.ab_forward_slice(p, bh0, nbh, Q, K, V, bufs)
+    barrier()
+    code = ab.device_error(dev)
+    if code:
+        raise SystemExit(f"device error during warm-up: {ab.status_string(code)}")
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    clocks.wait_first_sample()
+    barrier()
+    t0.record(stream)
+    for _ in range(args.steps):
+        ab.ab_forward_slice(p, bh0, nbh, Q, K, V, bufs)
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    code = ab.device_error(dev)
+    if code:
+        raise SystemExit(f"device error in the timed region: {ab.status_string(code)}")
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+
+    # end to end: each rank copies its slice in from pinned host memory, runs
+    # it, and copies its output back; the layer's bytes, the slowest rank's time
+    e2e = None
+    if not args.no_extras:
+        Qh, Kh, Vh = (t.pin_memory() for t in (Qs, Ks, Vs))
+        Oh = torch.empty_like(Qs).pin_memory()
+        steps = max(2, min(args.steps, 5))
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            Q.copy_(Qh, non_blocking=True)
+            K.copy_(Kh, non_blocking=True)
+            V.copy_(Vh, non_blocking=True)
+            ab.ab_forward_slice(p, bh0, nbh, Q, K, V, bufs)
+            Oh.copy_(bufs.O, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+        full = [t.numel() * t.element_size() for t in (Qc, Kc, Vc)]
+        e2e = {"value": round(dense_flop(w) / (ems * 1e-3) / 1e12, 3), "unit": UNIT,
+               "h2d_bytes_per_step": sum(full), "d2h_bytes_per_step": full[0], "ms_per_step": round(ems, 3),
+               "api": "ab_forward_slice with the slice's copies from pinned host memory on every rank"}
+    out = None
+    if rank == 0:
+        out = {"metric": METRIC, "value": round(dense_flop(w) / (ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+               "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+               "data": "synthetic",
+               "config": config_dict(w, {"parallelism": f"heads split over {world} GPUs "
+                                                        f"({[n for _, n in ab.head_slices(w.B, w.H, world)]} heads)"}),
+               "ms_per_layer": round(ms, 4), "gpu_launches": 5 * args.steps, "e2e": e2e, "clocks": clk}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
 def _select(ab, p, Q, K, bufs):
     import ctypes
     lib = ab.lib()
@@ -565,15 +662,20 @@ def run_reference(args):
     Qc, Kc, Vc = make_workload_qkv(w)
     for _ in range(args.warmup):  # untimed warm-up steps
         cpu_baseline(w, args, Qc, Kc, Vc)
-    vals = []
+    vals, walls = [], []
     last = None
     for _ in range(args.steps):
+        t = time.perf_counter()
         last = cpu_baseline(w, args, Qc, Kc, Vc)
+        walls.append(time.perf_counter() - t)
         vals.append(last["ms_per_layer_extrapolated"])
     ms = statistics.mean(vals)
     value = dense_flop(w) / (ms * 1e-3) / 1e12
     return {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": round(ms, 1),
+            "ms_per_step_kind": "extrapolated from the sampled units (wall x units per layer / sampled units)",
+            "ms_per_step_measured_wall": round(statistics.mean(walls) * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": config_dict(w, {"parallelism": "host threads"}),
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
@@ -595,12 +697,19 @@ def main():
     ap.add_argument("--kv-block", type=int, default=None, help="KV block size override (sweeps)")
     ap.add_argument("--keep", type=float, default=None, help="keep ratio override (sweeps)")
     ap.add_argument("--clusters", type=int, default=None, help="cluster count C override (sweeps)")
+    ap.add_argument("--split", choices=["replicas", "heads"], default="replicas",
+                    help="multi-GPU: one layer per GPU (replicas) or one layer's heads divided among the GPUs")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the end-to-end, dense and CPU-baseline legs (profiling only)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.impl == "reference":
+        out = run_reference(args)
+    elif args.split == "heads":
+        out = run_ours_split(args)
+    else:
+        out = run_ours(args)
     if out is not None:
         print(json.dumps(out), flush=True)
 

@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "AB_OK", 1: "AB_ERR_INVALID_ARG", 2: "AB_ERR_UNSUPPORTED", 3:
 # every symbol include/ab.h declares
 EXPORTS = ("ab_budget", "ab_workspace_size", "ab_select", "ab_sample", "ab_sample_systematic", "ab_sample_topk", "ab_attention",
            "ab_attention_dense", "ab_forward", "ab_forward_host", "ab_get_device_error",
-           "ab_status_string", "ab_select_static")
+           "ab_status_string", "ab_select_static", "ab_forward_slice")
 
 
 class AbError(RuntimeError):
@@ -111,13 +111,16 @@ def lib(path: str = LIB_PATH):
         L.ab_attention_dense.argtypes = [P, vp, vp, vp, vp, vp]
         L.ab_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ab_forward_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.ab_forward_slice.argtypes = [P, ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                       vp]
         L.ab_select_static.argtypes = [P, vp, vp, vp, vp, vp, vp]
         L.ab_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
         L.ab_status_string.argtypes = [ctypes.c_int]
         L.ab_status_string.restype = ctypes.c_char_p
         for name in ("ab_workspace_size", "ab_select", "ab_sample", "ab_sample_systematic", "ab_sample_topk", "ab_attention",
                      "ab_attention_dense",
-                     "ab_forward", "ab_forward_host", "ab_get_device_error", "ab_select_static"):
+                     "ab_forward", "ab_forward_host", "ab_get_device_error", "ab_select_static",
+                     "ab_forward_slice"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -283,6 +286,58 @@ def ab_forward(p: Params, Q, K, V, bufs: Buffers | None = None) -> Buffers:
     _check(lib().ab_forward(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(b.P), _ptr(b.idx),
                             _ptr(b.pi_q32), _ptr(b.count), _ptr(b.O), _ptr(b.ws), b.ws.numel(),
                             _stream(Q.device)), "ab_forward")
+    return b
+
+
+def head_slices(B: int, H: int, world: int):
+    """Contiguous near-equal partition of a layer's B * H heads among `world`
+    ranks: [(bh0, nbh), ...], rank r taking flattened heads [bh0, bh0 + nbh)
+    (the first B*H % world ranks take one head more).  Every rank gets at
+    least one head, so world must not exceed B * H."""
+    n = B * H
+    if not 1 <= world <= n:
+        raise ValueError(f"cannot split {n} heads among {world} ranks")
+    base, extra = divmod(n, world)
+    out, bh0 = [], 0
+    for r in range(world):
+        nbh = base + (1 if r < extra else 0)
+        out.append((bh0, nbh))
+        bh0 += nbh
+    return out
+
+
+def slice_rows(p: Params, bh0: int, nbh: int):
+    """(b, h, i) in the whole problem of every row of a slice's per-row
+    buffers (P, idx, pi_q32: [nbh, Nq, ...]; count: [nbh, Nq]), in their
+    order: local row r is row bh0 * Nq + r of the whole [B, H, Nq] layout.
+    These are the counters SIP draws a slice's rows with (the library derives
+    the same from the slice's first row and the whole problem's H)."""
+    out = []
+    for lb in range(nbh):
+        b, h = divmod(bh0 + lb, p.H)
+        out.extend((b, h, i) for i in range(p.Nq))
+    return out
+
+
+def slice_params(p: Params, nbh: int) -> Params:
+    """The problem of one slice of nbh heads (B = 1, H = nbh): its buffer
+    shapes and workspace size.  The whole problem's Params stay the ones
+    passed to ab_forward_slice."""
+    from dataclasses import replace
+    return replace(p, B=1, H=nbh)
+
+
+def ab_forward_slice(p: Params, bh0: int, nbh: int, Q, K, V, bufs: Buffers | None = None) -> Buffers:
+    """ab_forward on heads [bh0, bh0 + nbh) of the problem `p` (flattened b * H
+    + h): Q [1, nbh, L, d], K and V [1, nbh, Lk, d]; the buffers are the
+    slice's (Buffers(slice_params(p, nbh))).  The draws use the whole
+    problem's counters, so the result equals those heads of ab_forward(p)."""
+    ps = slice_params(p, nbh)
+    _check_qkv(ps, Q, K, V)
+    b = Buffers(ps, Q.device) if bufs is None else bufs
+    _check(lib().ab_forward_slice(ctypes.byref(p.c()), int(bh0), int(nbh), _ptr(Q), _ptr(K), _ptr(V), _ptr(b.P),
+                                  _ptr(b.idx), _ptr(b.pi_q32), _ptr(b.count), _ptr(b.O), _ptr(b.ws), b.ws.numel(),
+                                  _stream(Q.device)), "ab_forward_slice")
     return b
 
 

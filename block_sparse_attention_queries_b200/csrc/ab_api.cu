@@ -10,6 +10,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "ab_attention.cuh"
 #include "ab_sample.cuh"
@@ -27,6 +28,13 @@ struct Dims {
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// NVTX range around one entry point (host side: argument checks and launches);
+// free unless a profiler is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 int budget_of(int Nkv, double keep) {
   double kb = std::floor(keep * double(Nkv) + 0.5);
@@ -376,6 +384,7 @@ ab_status ab_workspace_size(const ab_params* p, size_t* bytes) {
 ab_status ab_select(const ab_params* p, const void* Q, const void* K, float* P, float* centroids, int32_t* counts,
                     void* workspace, size_t ws_bytes, void* stream) {
   Dims d;
+  NvtxRange nvtx("ab_select");
   const ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   return do_select(d, Q, K, P, centroids, counts, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
@@ -384,6 +393,7 @@ ab_status ab_select(const ab_params* p, const void* Q, const void* K, float* P, 
 ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,
                     void* stream) {
   Dims d;
+  NvtxRange nvtx("ab_sample");
   const ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   return do_sample(d, P, idx, pi_q32, count, static_cast<cudaStream_t>(stream));
@@ -392,6 +402,7 @@ ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* 
 ab_status ab_sample_systematic(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,
                                void* stream) {
   Dims d;
+  NvtxRange nvtx("ab_sample_systematic");
   const ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   if (!P || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
@@ -419,6 +430,7 @@ ab_status ab_sample_systematic(const ab_params* p, const float* P, int32_t* idx,
 ab_status ab_sample_topk(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,
                          void* stream) {
   Dims d;
+  NvtxRange nvtx("ab_sample_topk");
   const ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   if (!P || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
@@ -433,6 +445,7 @@ ab_status ab_sample_topk(const ab_params* p, const float* P, int32_t* idx, uint3
 ab_status ab_attention(const ab_params* p, const void* Q, const void* K, const void* V, const int32_t* idx,
                        const uint32_t* pi_q32, const int32_t* count, void* O, void* stream) {
   Dims d;
+  NvtxRange nvtx("ab_attention");
   const ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   return do_attention(d, Q, K, V, idx, pi_q32, count, O, false, static_cast<cudaStream_t>(stream));
@@ -441,6 +454,7 @@ ab_status ab_attention(const ab_params* p, const void* Q, const void* K, const v
 ab_status ab_attention_dense(const ab_params* p, const void* Q, const void* K, const void* V, void* O,
                              void* stream) {
   Dims d;
+  NvtxRange nvtx("ab_attention_dense");
   const ab_status s = check_params(p, false, &d);
   if (s != AB_OK) return s;
   return do_attention(d, Q, K, V, nullptr, nullptr, nullptr, O, true, static_cast<cudaStream_t>(stream));
@@ -449,6 +463,7 @@ ab_status ab_attention_dense(const ab_params* p, const void* Q, const void* K, c
 ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const void* V, float* P, int32_t* idx,
                      uint32_t* pi_q32, int32_t* count, void* O, void* workspace, size_t ws_bytes, void* stream) {
   Dims d;
+  NvtxRange nvtx("ab_forward");
   ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   if (!V || !O || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
@@ -458,6 +473,27 @@ ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const voi
   s = do_sample(d, P, idx, pi_q32, count, st);
   if (s != AB_OK) return s;
   return do_attention(d, Q, K, V, idx, pi_q32, count, O, false, st);
+}
+
+ab_status ab_forward_slice(const ab_params* p, int32_t bh0, int32_t nbh, const void* Q, const void* K,
+                           const void* V, float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count, void* O,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  NvtxRange nvtx("ab_forward_slice");
+  ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  if (nbh < 1 || bh0 < 0 || int64_t(bh0) + nbh > int64_t(d.BH)) return AB_ERR_INVALID_ARG;
+  if (!V || !O || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the slice as a problem of its own (B = 1, H = nbh); the draws keep the
+  // whole problem's counters (its H and the slice's first row)
+  Dims dc = d;
+  dc.B = 1; dc.H = nbh; dc.BH = nbh;
+  s = do_select(dc, Q, K, P, nullptr, nullptr, workspace, ws_bytes, st);
+  if (s != AB_OK) return s;
+  s = do_sample(dc, P, idx, pi_q32, count, st, d.H, int64_t(bh0) * d.Nq);
+  if (s != AB_OK) return s;
+  return do_attention(dc, Q, K, V, idx, pi_q32, count, O, false, st);
 }
 
 namespace {
@@ -484,6 +520,7 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
                           void* O_host, void* Q, void* K, void* V, float* P, int32_t* idx, uint32_t* pi_q32,
                           int32_t* count, void* O, void* workspace, size_t ws_bytes, void* stream) {
   Dims d;
+  NvtxRange nvtx("ab_forward_host");
   ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   if (!Q_host || !K_host || !V_host || !O_host || !Q || !K || !V || !O || !idx || !pi_q32 || !count)
@@ -559,6 +596,7 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
 ab_status ab_select_static(const ab_params* p, const void* Q, const void* K, float* P, float* centroids,
                            int32_t* counts, void* stream) {
   Dims d;
+  NvtxRange nvtx("ab_select_static");
   const ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   if (workspace_layout(d).total > size_t(AB_SELECT_STATIC_SCRATCH_BYTES)) return AB_ERR_WORKSPACE;

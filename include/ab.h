@@ -220,6 +220,25 @@ ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const voi
                      size_t ws_bytes, void* stream);
 
 /*
+ * ab_forward on a slice of the problem's heads: the (b, h) pairs whose
+ * flattened index b * H + h lies in [bh0, bh0 + nbh), for instance one GPU's
+ * share when a layer's heads are divided among GPUs.  Every (b, h) is
+ * independent on the whole path (selection, sampling and attention of a head
+ * read only that head's Q, K and V), so the slices need no exchange of data.
+ * *p describes the WHOLE problem (B, H and the rest); Q, O ([nbh, L, d]), K,
+ * V ([nbh, Lk, d]), P, idx, pi_q32 ([nbh, Nq, Nkv]) and count ([nbh, Nq])
+ * hold the slice only, in the layouts of the full tensors.  SIP's draws take
+ * the whole problem's counters (b, h, i, j), so the slice's lists and output
+ * are bit-identical to the same heads of ab_forward on the whole problem.
+ * `workspace` as for ab_select, sized for the slice (ab_workspace_size of
+ * the problem with B = 1, H = nbh).  AB_ERR_INVALID_ARG if the range is
+ * empty or leaves [0, B * H).
+ */
+ab_status ab_forward_slice(const ab_params* p, int32_t bh0, int32_t nbh, const void* Q, const void* K,
+                           const void* V, float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count, void* O,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * ab_forward from HOST buffers: copies Q_host (host, [B, H, L, d] bf16),
  * K_host and V_host (host, [B, H, Lk, d] bf16; page-locked memory gives
  * asynchronous copies) to the device buffers Q, K, V, runs the path, and

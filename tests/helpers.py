@@ -68,3 +68,24 @@ def oracle_sip_rows(P, Kb, seed, rows, threads=None):
         b, h, i = u
         return u, oracle.sip_row(P[b, h, i], Kb, seed, b, h, i)
     return dict(oracle.run_units(one, list(rows), threads))
+
+
+def selection_agreement(pairs, what=""):
+    """Selection of the CUDA path vs the oracle's, aggregated over rows:
+    pairs = [(gpu kept blocks, oracle kept blocks), ...].  Asserts and returns
+    (agreement, jaccard): agreement = sum |S_gpu & S_oracle| / sum |S_oracle|
+    >= 0.995 (the parity contract) and the Jaccard index sum |S_gpu & S_oracle|
+    / sum |S_gpu | S_oracle| >= 0.99 (both draws use the same uniforms, so the
+    two sets differ only at blocks whose inclusion probability the two
+    estimates put on different sides of the draw)."""
+    inter = tot = union = 0
+    for g, o in pairs:
+        a, b = set(np.asarray(g).tolist()), set(np.asarray(o).tolist())
+        inter += len(a & b)
+        tot += len(b)
+        union += len(a | b)
+    agree, jac = inter / max(tot, 1), inter / max(union, 1)
+    print(f"selection {what}: agreement {agree:.5f}, Jaccard {jac:.5f} over {len(pairs)} rows")
+    assert agree >= 0.995, (what, agree)
+    assert jac >= 0.99, (what, jac)
+    return agree, jac

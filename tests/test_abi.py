@@ -125,3 +125,14 @@ def test_list_outputs_are_checked_before_any_call():
         ab._list_outputs(p, P, (good[0].float(), good[1], good[2]))
     with pytest.raises(ValueError):
         ab._list_outputs(p, P.double(), good)
+
+
+def test_forward_slice_range_checked_on_host(lib):
+    # a slice must be a non-empty range of the whole problem's B * H heads;
+    # rejected before anything touches the device (pointers never read)
+    p = ab.Params(B=2, H=3, L=256, d=64, q_block=64, kv_block=16, C=4).c()
+    good = ctypes.c_void_p(0x1000)
+    args = (good,) * 8 + (good, ctypes.c_size_t(1 << 30), None)
+    for bh0, nbh in ((0, 0), (-1, 2), (5, 2), (0, 7)):
+        assert lib.ab_forward_slice(ctypes.byref(p), bh0, nbh, *args) == 1
+    assert lib.ab_forward_slice(ctypes.byref(p), 0, 2, good, good, None, *args[3:]) == 1  # V missing

@@ -21,8 +21,7 @@ import numpy as np
 import pytest
 
 import oracle
-from helpers import (assert_close_attention, np32, oracle_dense_units, oracle_ht_units, oracle_sip_rows,
-                     rel_l2)
+from helpers import (assert_close_attention, np32, oracle_dense_units, oracle_ht_units, oracle_sip_rows, rel_l2, selection_agreement)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -85,15 +84,12 @@ def test_cross_attention_end_to_end(dev, wname):
     # the sampler on the GPU's P, bit for bit; agreement with the oracle's selection
     sg = oracle_sip_rows(Pg, Kb, p.seed, units)
     so = oracle_sip_rows(Po.astype(np.float32), Kb, p.seed, units)
-    inter = tot = 0
     for r in units:
         c = int(gc[r])
         assert c == sg[r][2], (wname, r)
         np.testing.assert_array_equal(gi[r][:c], sg[r][0])
         np.testing.assert_array_equal(gp[r][:c], sg[r][1])
-        inter += len(set(gi[r][:c].tolist()) & set(so[r][0].tolist()))
-        tot += len(so[r][0])
-    assert inter / tot >= 0.995, (wname, inter / tot)
+    selection_agreement([(gi[r][:int(gc[r])], so[r][0]) for r in units], wname)
 
     # sparse attention on the GPU's lists
     ref = _stack(p, oracle_ht_units(Qn, Kn, Vn, p.q_block, p.kv_block, units, gi, gp, gc), units)
