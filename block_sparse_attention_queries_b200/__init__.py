@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "AB_OK", 1: "AB_ERR_INVALID_ARG", 2: "AB_ERR_UNSUPPORTED", 3:
 # every symbol include/ab.h declares
 EXPORTS = ("ab_budget", "ab_workspace_size", "ab_select", "ab_sample", "ab_sample_systematic", "ab_sample_topk", "ab_attention",
            "ab_attention_dense", "ab_forward", "ab_forward_host", "ab_get_device_error",
-           "ab_status_string", "ab_select_static", "ab_forward_slice")
+           "ab_status_string", "ab_select_static", "ab_forward_slice", "ab_select_sample")
 
 
 class AbError(RuntimeError):
@@ -111,6 +111,7 @@ def lib(path: str = LIB_PATH):
         L.ab_attention_dense.argtypes = [P, vp, vp, vp, vp, vp]
         L.ab_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ab_forward_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.ab_select_sample.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ab_forward_slice.argtypes = [P, ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                        vp]
         L.ab_select_static.argtypes = [P, vp, vp, vp, vp, vp, vp]
@@ -120,7 +121,7 @@ def lib(path: str = LIB_PATH):
         for name in ("ab_workspace_size", "ab_select", "ab_sample", "ab_sample_systematic", "ab_sample_topk", "ab_attention",
                      "ab_attention_dense",
                      "ab_forward", "ab_forward_host", "ab_get_device_error", "ab_select_static",
-                     "ab_forward_slice"):
+                     "ab_forward_slice", "ab_select_sample"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -222,6 +223,27 @@ def _lists_call(fn_name, p: Params, P, out=None):
     _check(getattr(lib(), fn_name)(ctypes.byref(p.c()), _ptr(P), _ptr(idx), _ptr(piq), _ptr(cnt),
                                    _stream(P.device)), fn_name)
     return idx, piq, cnt
+
+
+def ab_select_sample(p: Params, Q, K, workspace=None, out=None):
+    """ab_select then ab_sample in one call (the scoring kernel samples the
+    rows it scores when rows have at most 2048 KV blocks); returns
+    (P, idx, pi_q32, count), bit-identical to the two calls in a row.
+    `out` = (P, idx, pi_q32, count) writes into caller-owned tensors."""
+    import torch
+    _check_qkv(p, Q, K)
+    if out is None:
+        P = torch.empty(p.B, p.H, p.Nq, p.Nkv, dtype=torch.float32, device=Q.device)
+        idx, piq, cnt = _list_outputs(p, P, None)
+    else:
+        P, idx, piq, cnt = out
+        if P.dtype != torch.float32 or tuple(P.shape) != (p.B, p.H, p.Nq, p.Nkv) or not P.is_contiguous():
+            raise ValueError("P must be contiguous float32 [B, H, Nq, Nkv]")
+        idx, piq, cnt = _list_outputs(p, P, (idx, piq, cnt))
+    ws = alloc_workspace(p, Q.device) if workspace is None else workspace
+    _check(lib().ab_select_sample(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(P), _ptr(idx), _ptr(piq), _ptr(cnt),
+                                  _ptr(ws), ws.numel(), _stream(Q.device)), "ab_select_sample")
+    return P, idx, piq, cnt
 
 
 def ab_sample(p: Params, P, out=None):

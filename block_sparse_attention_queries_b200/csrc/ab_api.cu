@@ -146,9 +146,11 @@ ab_status launch_status() {
 }
 
 // ---------------------------------------------------------------- launches
+// sip != nullptr: the scoring kernel also runs SIP on its rows (rows of at
+// most kFusedSampleMaxNkv blocks).
 template <int D>
 ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, float* cent, int32_t* counts,
-                     uint8_t* ws, cudaStream_t st) {
+                     uint8_t* ws, cudaStream_t st, const SipArgs* sip = nullptr) {
   const Workspace w = workspace_layout(d);
   auto* ksum = reinterpret_cast<__nv_bfloat16*>(ws + w.off_ksum);
   auto* cent_ws = reinterpret_cast<__nv_bfloat16*>(ws + w.off_cent);
@@ -194,6 +196,7 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, floa
     a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
     const int n_last = d.Lk - (d.Nkv - 1) * d.kv_block;
     a.last_bias = float(std::log2(double(n_last) / double(d.kv_block)));
+    if (sip) a.sip = *sip;
     const int G = 128 / d.C;
     const unsigned grid = unsigned(d.BH * ((d.Nq + G - 1) / G));
     const int smem = ScSmem<D>::kAlloc;
@@ -202,6 +205,15 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, floa
       kern<<<grid, 288, smem, st>>>(tmCent, tmKsum, a);
       return launch_status();
     };
+    if (sip) {
+      switch (d.C) {
+        case 1: return launch(score_kernel<D, 1, true>);
+        case 2: return launch(score_kernel<D, 2, true>);
+        case 4: return launch(score_kernel<D, 4, true>);
+        case 8: return launch(score_kernel<D, 8, true>);
+        default: return launch(score_kernel<D, 16, true>);
+      }
+    }
     switch (d.C) {
       case 1: return launch(score_kernel<D, 1>);
       case 2: return launch(score_kernel<D, 2>);
@@ -299,6 +311,32 @@ ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q3
   return launch_status();
 }
 
+constexpr int kFusedSampleMaxNkv = 2048;  // rows the scoring kernel's warps sample in registers
+
+// ab_select then ab_sample; for rows of at most kFusedSampleMaxNkv blocks in
+// one launch less (the scoring kernel samples the rows it has just scored).
+// H and row0 as for do_sample.
+ab_status do_select_sample(const Dims& d, const void* Q, const void* K, float* P, int32_t* idx, uint32_t* pi_q32,
+                           int32_t* count, void* ws, size_t ws_bytes, cudaStream_t st, int H = -1,
+                           int64_t row0 = 0) {
+  if (d.Nkv > kFusedSampleMaxNkv) {
+    const ab_status s = do_select(d, Q, K, P, nullptr, nullptr, ws, ws_bytes, st);
+    return s != AB_OK ? s : do_sample(d, P, idx, pi_q32, count, st, H, row0);
+  }
+  if (!Q || !K || !P || !ws || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(P) || !aligned16(ws)) return AB_ERR_INVALID_ARG;
+  if (!aligned16(idx) || !aligned16(pi_q32) || !aligned16(count)) return AB_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_layout(d).total) return AB_ERR_WORKSPACE;
+  SipArgs a{};
+  a.P = P; a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
+  a.H = H > 0 ? H : d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
+  a.seed_lo = uint32_t(d.seed); a.seed_hi = uint32_t(d.seed >> 32);
+  a.row0 = row0;
+  auto* w = reinterpret_cast<uint8_t*>(ws);
+  return d.d == 128 ? run_select<128>(d, Q, K, P, nullptr, nullptr, w, st, &a)
+                    : run_select<64>(d, Q, K, P, nullptr, nullptr, w, st, &a);
+}
+
 ab_status do_attention(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* idx,
                        const uint32_t* pi_q32, const int32_t* count, void* O, bool dense, cudaStream_t st) {
   if (!Q || !K || !V || !O) return AB_ERR_INVALID_ARG;
@@ -388,6 +426,15 @@ ab_status ab_select(const ab_params* p, const void* Q, const void* K, float* P, 
   const ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   return do_select(d, Q, K, P, centroids, counts, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+ab_status ab_select_sample(const ab_params* p, const void* Q, const void* K, float* P, int32_t* idx,
+                           uint32_t* pi_q32, int32_t* count, void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  const ab_status s = check_params(p, true, &d);
+  if (s != AB_OK) return s;
+  NvtxRange nvtx("ab_select_sample");
+  return do_select_sample(d, Q, K, P, idx, pi_q32, count, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 ab_status ab_sample(const ab_params* p, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count,

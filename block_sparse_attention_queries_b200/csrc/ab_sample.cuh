@@ -340,12 +340,16 @@ __global__ void __launch_bounds__(kSipThreads) sip_kernel(const SipArgs a) {
 // the same Pi (as systematic_pass: one offset U per row, block j kept iff a
 // point U + m 2^32 lies in [C_j, C_j + Pi_j), C_j the running sum of Pi in
 // ascending j, here a warp scan per 128-block chunk).
-template <int KMAX, bool kSystematic>
-__global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows) {
+// One warp samples row `row` of a.P (Nkv <= 128 KMAX), the whole row's
+// quantised weights in registers (KMAX x 4 per lane).  kCoherent: P was
+// written earlier by the calling kernel itself, so it is read through L2
+// (__ldcg) rather than the read-only path, which is only valid for data the
+// kernel does not write.
+template <int KMAX, bool kSystematic, bool kCoherent>
+__device__ __forceinline__ void sip_warp_row(const SipArgs& a, int row) {
   static_assert(KMAX * 4 * 16777216ull < 4294967296ull, "per-lane partial sums must fit 32 bits");
   const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= rows) return;  // whole warp: no block-level synchronisation below
+  auto loadP = [](const float* p) { return kCoherent ? __ldcg(p) : __ldg(p); };
   const int64_t grow = a.row0 + row;
   const int b = int(grow / (int64_t(a.H) * a.Nq));
   const int h = int((grow / a.Nq) % a.H);
@@ -358,7 +362,7 @@ __global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int j = 128 * k + 4 * lane + q;
-      w[k][q] = j < Nkv ? quantise_w(__ldg(P + j)) : 0u;  // entries >= Nkv: 0, never capped
+      w[k][q] = j < Nkv ? quantise_w(loadP(P + j)) : 0u;  // entries >= Nkv: 0, never capped
     }
   }
 
@@ -491,10 +495,18 @@ __global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows
   // ---- inclusion probabilities of the kept entries (as in sip_kernel)
   for (int e = lane; e < base; e += 32) {
     const int j = out_idx[e];
-    const uint32_t wj = quantise_w(__ldg(P + j));
+    const uint32_t wj = quantise_w(loadP(P + j));
     out_pi[e] = wj < theta ? pi_free(uint64_t(R32) * wj, S_hi, S_lo, inv_s32) : 0u;
   }
   if (lane == 0) a.count[row] = base;
+}
+
+// One warp per row for rows of at most 128 KMAX blocks.
+template <int KMAX, bool kSystematic>
+__global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;  // whole warp: no block-level synchronisation below
+  sip_warp_row<KMAX, kSystematic, false>(a, row);
 }
 
 // Truncation, the selection SIP is contrasted with (AB-Attention page,

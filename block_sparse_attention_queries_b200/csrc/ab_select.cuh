@@ -23,6 +23,7 @@
 #pragma once
 
 #include "ab_ptx.cuh"
+#include "ab_sample.cuh"
 
 namespace ab {
 
@@ -355,6 +356,7 @@ struct ScoreArgs {
   float* P;                  // [BH, Nq, Nkv]
   float scale_log2;          // log2(e) / sqrt(d)
   float last_bias;           // log2(n_last / kv_block) of the last KV block
+  SipArgs sip;               // kSample: SIP of the CTA's rows right after their P (P = sip.P rows)
 };
 
 // Reduce 32 per-lane values over aligned groups of C lanes and scatter the
@@ -381,7 +383,12 @@ __device__ __forceinline__ void group_reduce_scatter(float (&v)[32], int lane) {
 // [64 (w / 4), +64) of every 128-column chunk), warp 8 loads and issues the
 // MMAs.  Two CTAs share an SM (96 KB of shared memory, 256 TMEM columns each).  The two column halves of a row keep separate running max / sum in
 // the first pass and merge them before the second.
-template <int D, int C>
+// kSample (rows of at most 2048 blocks): once the CTA's rows of P are written,
+// its nine warps run SIP on them (sip_warp_row, one warp per row), so the
+// sampling of these rows starts as soon as their estimate exists, next to the
+// scoring of the other CTAs, without a second launch or a DRAM round trip of
+// P (it is read back from L2).
+template <int D, int C, bool kSample = false>
 __global__ void __launch_bounds__(288, 2)
     score_kernel(const __grid_constant__ CUtensorMap tmCent, const __grid_constant__ CUtensorMap tmKsum,
                  const ScoreArgs a) {
@@ -562,11 +569,20 @@ __global__ void __launch_bounds__(288, 2)
       }
     }
   }
+  if constexpr (kSample) __threadfence();  // P visible in L2 to the sampling warps below
   tc_fence_before();
   __syncthreads();
   if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
+  }
+  if constexpr (kSample) {
+    if (!*abort_flag) {
+      for (int r = warp; r < G; r += 9) {
+        const int i = i0 + r;
+        if (i < a.Nq) sip_warp_row<16, false, true>(a.sip, bh * a.Nq + i);
+      }
+    }
   }
 }
 

@@ -211,6 +211,21 @@ ab_status ab_attention_dense(const ab_params* p, const void* Q, const void* K, c
                              void* stream);
 
 /*
+ * ab_select followed by ab_sample, with the same outputs (P and the lists,
+ * bit-identical to the two calls in a row), in one launch less: for rows of
+ * at most 2048 KV blocks the scoring kernel runs SIP on the rows of P it has
+ * just computed (AB-Attention page, "AB-Attention ve Üç Temel Yeniliği": the
+ * IBCS estimate is what SIP samples from), so P is read back from L2 rather
+ * than after a DRAM round trip.  Longer rows run the two steps as separate
+ * launches.  Arguments as for ab_select (P is still written) and ab_sample;
+ * errors as for those two calls.  On a B200 the fused launch measured slower
+ * than the two launches (its nine warps per scoring CTA sample with fewer
+ * rows in flight than the sampler's own grid), so ab_forward keeps the two.
+ */
+ab_status ab_select_sample(const ab_params* p, const void* Q, const void* K, float* P, int32_t* idx,
+                           uint32_t* pi_q32, int32_t* count, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * The three steps in order on device buffers: ab_select (into P, with
  * centroids/counts not kept), ab_sample, ab_attention.  `workspace` as for
  * ab_select.
