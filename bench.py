@@ -391,6 +391,8 @@ def run_ours(args):
         else:
             dense_ms = run_dense(ab, p, Q, K, V, dev, 3)
             qual = quality(ab, p, Q, K, V, bufs, dev)
+            qual["ms_select_sample_fused"] = time_fused_select_sample(ab, p, Q, K, dev)
+            qual["concentrated"] = quality_concentrated(ab, w, dev)
             cpu = cpu_baseline(w, args, Qc, Kc, Vc)
         out = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -605,6 +607,50 @@ def quality(ab, p, Q, K, V, bufs, dev):
             "ms_sample_systematic": round(t2.elapsed_time(t3) / 3, 4),
             "ms_sample_truncation": round(t0.elapsed_time(t1) / 3, 4),
             "note": "same P and budget; information only, not a gate"}
+
+
+def time_fused_select_sample(ab, p, Q, K, dev, iters=3):
+    """ab_select_sample (scoring that samples the rows it scores) on the same
+    inputs, into preallocated outputs: information beside ms_select + ms_sample."""
+    import torch
+    ws = ab.alloc_workspace(p, dev)
+    out = ab.ab_select_sample(p, Q, K, workspace=ws)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(iters):
+        ab.ab_select_sample(p, Q, K, workspace=ws, out=out)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    return round(t0.elapsed_time(t1) / iters, 4)
+
+
+def quality_concentrated(ab, w, dev, heads=8, s_peak=32.0):
+    """Information only: the relative L2 distance to dense attention of SIP,
+    systematic sampling and truncation at the same budget when attention is
+    concentrated (inputs drawn with s_peak = 32 instead of 8, so that q.k /
+    sqrt(d) of two tokens at the same position is about 32: a few blocks hold
+    most of each row's weight), on the first `heads` heads of the workload."""
+    import torch
+    from block_sparse_attention_queries_b200.synthetic import make_qkv
+    wc = w.with_(H=min(heads, w.H))
+    p = ab.Params.of(wc, seed=42)
+    Qc, Kc, Vc = make_qkv(wc.B, wc.H, wc.grid, wc.d, wc.F, s_peak=s_peak)
+    Q, K, V = (t.to(dev) for t in (Qc, Kc, Vc))
+    b = ab.ab_forward(p, Q, K, V)
+    Od = ab.ab_attention_dense(p, Q, K, V)
+    Ot = ab.ab_attention(p, Q, K, V, *ab.ab_sample_topk(p, b.P))
+    Os = ab.ab_attention(p, Q, K, V, *ab.ab_sample_systematic(p, b.P))
+    torch.cuda.synchronize(dev)
+    ref = torch.linalg.vector_norm(Od.double())
+
+    def rel(o):
+        return round(float(torch.linalg.vector_norm(o.double() - Od.double()) / ref), 5)
+
+    return {"s_peak": s_peak, "heads": wc.H, "rel_l2_sip_vs_dense": rel(b.O),
+            "rel_l2_systematic_vs_dense": rel(Os), "rel_l2_truncation_vs_dense": rel(Ot),
+            "kept_block_fraction": round(float(b.count.sum()) / (wc.B * wc.H * wc.Nq * wc.Nkv), 5)}
 
 
 # ---------------------------------------------------------- CPU oracle arm

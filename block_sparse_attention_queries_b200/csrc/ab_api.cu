@@ -545,21 +545,48 @@ ab_status ab_forward_slice(const ab_params* p, int32_t bh0, int32_t nbh, const v
 
 namespace {
 
-// Streams and events of one pipelined host call, released on every path.
+// Copy streams and events of the pipelined host call, created on a
+// context's first call and kept for the library's lifetime (one set per
+// CUDA context, like the static scratch address).  A call holds the set's
+// lock while it enqueues, so calls from several host threads take turns;
+// re-recording an event after a stream has waited on it is safe (the wait
+// captured the earlier record).
 struct HostPipe {
+  CUcontext ctx = nullptr;
   cudaStream_t in = nullptr, out = nullptr;
-  std::vector<cudaEvent_t> ev;
-  ~HostPipe() {
-    for (cudaEvent_t e : ev) cudaEventDestroy(e);  // released once their work completes
-    if (in) cudaStreamDestroy(in);
-    if (out) cudaStreamDestroy(out);
-  }
-  bool event(cudaEvent_t* e) {
-    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
-    ev.push_back(*e);
-    return true;
-  }
+  cudaEvent_t start = nullptr, done = nullptr, in_done = nullptr, comp_done = nullptr;
+  std::mutex mu;
 };
+std::mutex g_pipes_mutex;
+std::vector<HostPipe*> g_pipes;  // never freed: streams outlive every call
+
+HostPipe* host_pipe_current_context() {
+  auto get_ctx = ctx_current_fn();
+  if (!get_ctx) return nullptr;
+  CUcontext ctx = nullptr;
+  int dev = -1;  // setting the current device makes its primary context current if none was
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
+  std::lock_guard<std::mutex> lock(g_pipes_mutex);
+  for (HostPipe* h : g_pipes)
+    if (h->ctx == ctx) return h;
+  HostPipe* h = new HostPipe;
+  h->ctx = ctx;
+  cudaEvent_t* evs[4] = {&h->start, &h->done, &h->in_done, &h->comp_done};
+  bool ok = cudaStreamCreateWithFlags(&h->in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&h->out, cudaStreamNonBlocking) == cudaSuccess;
+  for (cudaEvent_t* e : evs) ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    for (cudaEvent_t* e : evs)
+      if (*e) cudaEventDestroy(*e);
+    if (h->in) cudaStreamDestroy(h->in);
+    if (h->out) cudaStreamDestroy(h->out);
+    delete h;
+    return nullptr;
+  }
+  g_pipes.push_back(h);
+  return h;
+}
 
 }  // namespace
 
@@ -592,12 +619,12 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
   }
   // Pipelined over groups of heads (every (b, h) is independent): the inputs
   // of group c + 1 cross PCIe while group c computes on the caller's stream
-  // and group c - 1's output crosses back, on two streams of this call.
-  HostPipe pipe;
-  if (cudaStreamCreateWithFlags(&pipe.in, cudaStreamNonBlocking) != cudaSuccess) return AB_ERR_CUDA;
-  if (cudaStreamCreateWithFlags(&pipe.out, cudaStreamNonBlocking) != cudaSuccess) return AB_ERR_CUDA;
-  cudaEvent_t start, done;
-  if (!pipe.event(&start) || !pipe.event(&done)) return AB_ERR_CUDA;
+  // and group c - 1's output crosses back, on the context's two copy streams.
+  HostPipe* hp = host_pipe_current_context();
+  if (!hp) return AB_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(hp->mu);
+  HostPipe& pipe = *hp;
+  const cudaEvent_t start = pipe.start, done = pipe.done, in_done = pipe.in_done, comp_done = pipe.comp_done;
   if (cudaEventRecord(start, st) != cudaSuccess) return AB_ERR_CUDA;  // after the caller's earlier work
   if (cudaStreamWaitEvent(pipe.in, start, 0) != cudaSuccess) return AB_ERR_CUDA;
   if (cudaStreamWaitEvent(pipe.out, start, 0) != cudaSuccess) return AB_ERR_CUDA;
@@ -607,8 +634,6 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
     const int nbh = per < d.BH - bh0 ? per : d.BH - bh0;
     const size_t off = size_t(bh0) * q_head, bytes = size_t(nbh) * q_head;           // Q, O
     const size_t koff = size_t(bh0) * kv_head, kbytes = size_t(nbh) * kv_head;       // K, V
-    cudaEvent_t in_done, comp_done;
-    if (!pipe.event(&in_done) || !pipe.event(&comp_done)) return AB_ERR_CUDA;
     if (cudaMemcpyAsync(bw(Q, off), bf(Q_host, off), bytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess ||
         cudaMemcpyAsync(bw(K, koff), bf(K_host, koff), kbytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess ||
         cudaMemcpyAsync(bw(V, koff), bf(V_host, koff), kbytes, cudaMemcpyHostToDevice, pipe.in) != cudaSuccess)

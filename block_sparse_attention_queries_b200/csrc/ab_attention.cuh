@@ -21,8 +21,10 @@
 //   O_s += P_s V         tcgen05 (A = P_s in TMEM, B = V in shared memory)
 // Weighting every term of block j by 1/pi_j is the additive bias log2(1/pi_j)
 // inside the exponent, so the weights enter the running max and sum for free.
-// The reference max m moves only when a row max passes it by more than 8
-// (factor 256); O_s is then rescaled in TMEM by the softmax warps themselves.
+// The reference max m moves only when a row max passes it by more than
+// kLazyMax (a factor 2^16: the bf16 weights stay far from overflow, and the
+// 1/pi biases, up to 32 in log2, move the max less often than with a tighter
+// bound); O_s is then rescaled in TMEM by the softmax warps themselves.
 //
 // The two streams ping-pong: while the softmax warps of one stream work, the
 // tensor core runs the other stream's MMAs.  The MMA warp issues, per tile of
@@ -60,44 +62,53 @@ struct AttnArgs {
 };
 
 constexpr int kAttnThreads = 384;
+constexpr float kLazyMax = 16.f;  // log2 slack of the lazily moved reference max
 constexpr int kRegsLaunch = 168;   // registers per thread the kernel is launched with
 constexpr int kRegsCtl = 56;       // producer / MMA warpgroup after re-balancing
 constexpr int kRegsSoftmax = 224;  // softmax warpgroups after re-balancing
 static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kAttnThreads * kRegsLaunch, "register split exceeds the launch");
+
+// Stages of the K and V tile rings.
+constexpr int kKRing = 3;
+constexpr int kVRing = 2;
+constexpr int kAttnBars = 13 + 2 * (kKRing + kVRing);  // mbarriers (listed below)
 
 template <int D>
 struct AttnSmem {
   static constexpr int kSlabs = D / 64;
   static constexpr int kSlab = 128 * 128;       // one 128-row x 128-byte slab
   static constexpr int kTile = kSlabs * kSlab;  // 128 rows x D bf16
-  static constexpr int kKStages = 3;
-  static constexpr int kVStages = 2;
+  static constexpr int kKStages = kKRing;
+  static constexpr int kVStages = kVRing;
   static constexpr int kOffQ = 0;  // two Q tiles
   static constexpr int kOffK = kOffQ + 2 * kTile;
   static constexpr int kOffV = kOffK + kKStages * kTile;
   static constexpr int kOffMeta = kOffV + kVStages * kTile;  // per K stage: 8 biases, 8 valid counts
   static constexpr int kMetaStride = 64;
   static constexpr int kOffBar = kOffMeta + kKStages * kMetaStride;
-  static constexpr int kNumBars = 23;
+  static constexpr int kNumBars = kAttnBars;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+  static_assert(kAlloc <= 232448, "more shared memory than a CTA may have");
 };
 
 // barrier indices
 enum : int {
-  kBarQ = 0,       // 2 (per stream)
-  kBarKFull = 2,   // 3
-  kBarKEmpty = 5,  // 3 (128 arrivals: the softmax warps of the tile's stream)
-  kBarVFull = 8,   // 2
-  kBarVEmpty = 10, // 2
-  kBarSFull = 12,  // 2 (per stream)
-  kBarPFull = 14,  // 2 (per stream, 128 arrivals)
-  kBarOFinal = 16, // 2 (per stream)
-  kBarDrain = 18,
-  kBarPHalf = 19,  // 2 (per stream, 128 arrivals): keys [0, 64) of P are in TMEM
-  kBarOStaged = 21,  // 2 (per stream, one arrival per warp): the output tile is in shared memory
+  kBarQ = 0,                          // 2 (per stream)
+  kBarKFull = 2,                      // kKRing
+  kBarKEmpty = kBarKFull + kKRing,    // kKRing (128 arrivals: the softmax warps of the tile's stream)
+  kBarVFull = kBarKEmpty + kKRing,    // kVRing
+  kBarVEmpty = kBarVFull + kVRing,    // kVRing
+  kBarSFull = kBarVEmpty + kVRing,    // 2 (per stream)
+  kBarPFull = kBarSFull + 2,          // 2 (per stream, 128 arrivals)
+  kBarOFinal = kBarPFull + 2,         // 2 (per stream)
+  kBarDrain = kBarOFinal + 2,
+  kBarPHalf = kBarDrain + 1,          // 2 (per stream, 128 arrivals): keys [0, 64) of P are in TMEM
+  kBarOStaged = kBarPHalf + 2,        // 2 (per stream, one arrival per warp): the output tile is in shared memory
+  kBarCount = kBarOStaged + 2,
 };
+static_assert(kBarCount == kAttnBars, "barrier count");
 
 // Warp-uniform bounded wait: every lane of the calling warp gets the same answer.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -181,23 +192,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const Merge mg(T[0], T[1]);
   const int G = mg.total();
   // Dense attention with two query blocks: both streams read the same K and V
-  // tiles (keys [128t, 128t+128)), so each is loaded once, into K stage t % 3
+  // tiles (keys [128t, 128t+128)), so each is loaded once, into K stage t % kKRing
   // and V stage t % 2, for merged tiles 2t and 2t+1; otherwise every merged
-  // tile g has stages of its own (g % 3, g % 2).
+  // tile g has stages of its own (g % kKRing, g % kVRing).
   const bool share = kDense && T[0] == T[1];
 
   if (threadIdx.x == 0) {
+    for (int k = 0; k < kVRing; ++k) {
+      mbar_init(bar(kBarVFull + k), 1);
+      mbar_init(bar(kBarVEmpty + k), 1);
+    }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarQ + s), 1);
-      mbar_init(bar(kBarVFull + s), 1);
-      mbar_init(bar(kBarVEmpty + s), 1);
       mbar_init(bar(kBarSFull + s), 1);
       mbar_init(bar(kBarPFull + s), 128);
       mbar_init(bar(kBarPHalf + s), 128);
       mbar_init(bar(kBarOFinal + s), 1);
       mbar_init(bar(kBarOStaged + s), 4);
     }
-    for (int k = 0; k < 3; ++k) {
+    for (int k = 0; k < kKRing; ++k) {
       mbar_init(bar(kBarKFull + k), 1);
       mbar_init(bar(kBarKEmpty + k), share ? 256 : 128);  // the softmax warps of every stream that reads it
     }
@@ -266,7 +279,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t pq_cur, pq_next, pq_far;
     fetch(0, j_cur, pq_cur);
     fetch(1, j_next, pq_next);
-    const int nstage = is_k ? 3 : 2;
+    const int nstage = is_k ? kKRing : kVRing;
     const uint32_t full0 = bar(is_k ? kBarKFull : kBarVFull), empty0 = bar(is_k ? kBarKEmpty : kBarVEmpty);
     const uint32_t dst0 = sbase + (is_k ? SM::kOffK : SM::kOffV);
     const CUtensorMap* tm = is_k ? &tmK : &tmV;
@@ -343,8 +356,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (T[s] > 0) ok = mbar_wait(bar(kBarQ + s), 0, abort_flag);
       auto issue_S = [&](int s, int t) -> bool {
         const int ki = share ? t : mg.index(s, t);
-        const int ks = ki % 3;
-        if (!mbar_wait(bar(kBarKFull + ks), (ki / 3) & 1, abort_flag)) return false;
+        const int ks = ki % kKRing;
+        if (!mbar_wait(bar(kBarKFull + ks), (ki / kKRing) & 1, abort_flag)) return false;
         tc_fence_after();
         // K tile: next 64 columns at kHalfK, 8-row groups kSboK apart
         constexpr uint32_t kHalfK = kGrouped ? 1024u : uint32_t(SM::kSlab);
@@ -373,14 +386,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // softmax warps have stored keys [0, 64) of P
         if (!mbar_wait(bar(kBarPHalf + s), t & 1, abort_flag)) { ok = false; break; }
         const int vi = share ? t : g;  // V tile's position in the V ring's loads
-        if (!mbar_wait(bar(kBarVFull + (vi & 1)), (vi >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(kBarVFull + vi % kVRing), (vi / kVRing) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tO = tmem + 256u + uint32_t(s * D);
         const uint32_t tP = tmem + uint32_t(s) * 128u;
         // V tile (MN-major): 16 keys per k-step, next 64 columns at kLboV, next 8 keys at kSboV
         constexpr uint32_t kStepV = kGrouped ? 16u * uint32_t(SM::kSlabs) * 128u : 2048u;
         SmemDesc vd = vdesc0;
-        vd.lo += uint32_t(vi & 1) * uint32_t(SM::kTile >> 4);
+        vd.lo += uint32_t(vi % kVRing) * uint32_t(SM::kTile >> 4);
         mma_bf16_ts(tO, tP, desc_at(vd, 0), idO, t > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 1; kk < 4; ++kk) mma_bf16_ts(tO, tP + uint32_t(kk * 8), desc_at(vd, kk * kStepV), idO, 1u);
@@ -388,7 +401,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 4; kk < 8; ++kk) mma_bf16_ts(tO, tP + uint32_t(kk * 8), desc_at(vd, kk * kStepV), idO, 1u);
-        if (!share || s == 1) mma_commit(bar(kBarVEmpty + (vi & 1)));  // shared: after both streams' P V
+        if (!share || s == 1) mma_commit(bar(kBarVEmpty + vi % kVRing));  // shared: after both streams' P V
         if (t + 1 < T[s]) {
           ok = issue_S(s, t + 1);
         } else {
@@ -441,9 +454,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       };
       const int ki = share ? t : mg.index(s, t);  // K tile's position in the K ring's loads
-      const int ks = ki % 3;
+      const int ks = ki % kKRing;
       if (!warp_wait(bar(kBarSFull + s), t & 1, abort_flag)) { ok = false; break; }
-      if (!warp_wait(bar(kBarKFull + ks), (ki / 3) & 1, abort_flag)) { ok = false; break; }
+      if (!warp_wait(bar(kBarKFull + ks), (ki / kKRing) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float x[128];
 #pragma unroll
@@ -478,7 +491,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mx = fmaxf(mx, x[e * KVB + KVB - 1]);
           rmax = fmaxf(rmax, fmaf(mx, a.scale_log2, s_bias[e]));
         }
-        need = rmax > m_use + 8.f;
+        need = rmax > m_use + kLazyMax;
         if (need) {
           alpha = ex2_approx(m_use - rmax);  // 0 on the first tile
           m_use = rmax;
@@ -511,8 +524,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           x[k] = (w < s_valid[e]) ? fmaf(x[k], a.scale_log2, s_bias[e]) : -INFINITY;
           rmax = fmaxf(rmax, x[k]);
         }
-        // lazy reference max: move it only when the row max passes it by > 8
-        need = rmax > m_use + 8.f;
+        // lazy reference max: move it only when the row max passes it by > kLazyMax
+        need = rmax > m_use + kLazyMax;
         if (need) {
           alpha = ex2_approx(m_use - rmax);  // 0 on the first tile
           m_use = rmax;

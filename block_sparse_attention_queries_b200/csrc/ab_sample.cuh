@@ -454,51 +454,51 @@ __device__ __forceinline__ void sip_warp_row(const SipArgs& a, int row) {
       base_c += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) a.count[row] = base;
-    return;
-  }
+  } else {
 #pragma unroll
-  for (int k = 0; k < KMAX; ++k) {
-    if (128 * k >= Nkv) break;  // warp-uniform
-    const int j0 = 128 * k + 4 * lane;
-    uint32_t keep_mask = 0;
-    if (j0 < Nkv) {
-      const uint4 u4 = philox4x32_10(make_uint4(uint32_t(j0 >> 2), uint32_t(i), uint32_t(h), uint32_t(b)),
-                                     a.seed_lo, a.seed_hi);
-      const uint32_t us[4] = {u4.x, u4.y, u4.z, u4.w};
+    for (int k = 0; k < KMAX; ++k) {
+      if (128 * k >= Nkv) break;  // warp-uniform
+      const int j0 = 128 * k + 4 * lane;
+      uint32_t keep_mask = 0;
+      if (j0 < Nkv) {
+        const uint4 u4 = philox4x32_10(make_uint4(uint32_t(j0 >> 2), uint32_t(i), uint32_t(h), uint32_t(b)),
+                                       a.seed_lo, a.seed_hi);
+        const uint32_t us[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        bool keep;
-        if (w[k][q] >= theta) {
-          keep = true;
-        } else {
-          const uint64_t X = uint64_t(R32) * w[k][q];
-          keep = us[q] == 0u || mul_le_shift32(us[q], S_hi, S_lo, X);
+        for (int q = 0; q < 4; ++q) {
+          bool keep;
+          if (w[k][q] >= theta) {
+            keep = true;
+          } else {
+            const uint64_t X = uint64_t(R32) * w[k][q];
+            keep = us[q] == 0u || mul_le_shift32(us[q], S_hi, S_lo, X);
+          }
+          if (keep && j0 + q < Nkv) keep_mask |= 1u << q;
         }
-        if (keep && j0 + q < Nkv) keep_mask |= 1u << q;
       }
-    }
-    const int mine = __popc(keep_mask);
-    int incl = mine;
+      const int mine = __popc(keep_mask);
+      int incl = mine;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int pos = base + incl - mine;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int pos = base + incl - mine;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (keep_mask & (1u << q)) out_idx[pos++] = j0 + q;
-    base += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  __syncwarp();  // out_idx written by the other lanes is read below
+      for (int q = 0; q < 4; ++q)
+        if (keep_mask & (1u << q)) out_idx[pos++] = j0 + q;
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncwarp();  // out_idx written by the other lanes is read below
 
-  // ---- inclusion probabilities of the kept entries (as in sip_kernel)
-  for (int e = lane; e < base; e += 32) {
-    const int j = out_idx[e];
-    const uint32_t wj = quantise_w(loadP(P + j));
-    out_pi[e] = wj < theta ? pi_free(uint64_t(R32) * wj, S_hi, S_lo, inv_s32) : 0u;
+    // ---- inclusion probabilities of the kept entries (as in sip_kernel)
+    for (int e = lane; e < base; e += 32) {
+      const int j = out_idx[e];
+      const uint32_t wj = quantise_w(loadP(P + j));
+      out_pi[e] = wj < theta ? pi_free(uint64_t(R32) * wj, S_hi, S_lo, inv_s32) : 0u;
+    }
+    if (lane == 0) a.count[row] = base;
   }
-  if (lane == 0) a.count[row] = base;
 }
 
 // One warp per row for rows of at most 128 KMAX blocks.

@@ -38,15 +38,15 @@
  *    (Nkv = ceil(Lk / kv_block)); the last block of each kind may be
  *    partial.
  *  - Memory: the caller allocates and owns every buffer (device memory unless a
- *    call says "host"); the library allocates and frees no memory (only a
- *    pipelined ab_forward_host call creates, and releases, two streams and
- *    their events).
+ *    call says "host"); the library allocates and frees no memory (the
+ *    pipelined ab_forward_host creates two copy streams and four events per
+ *    CUDA context on its first call and keeps them).
  *    Every device pointer must be 16-byte aligned.
  *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  *    Every call only enqueues work on it and returns; results are ready when
  *    the stream reaches them.  The library keeps no state between calls other
- *    than the device error word and the fixed scratch array behind
- *    ab_select_static.
+ *    than the device error word, the fixed scratch array behind
+ *    ab_select_static and ab_forward_host's copy streams.
  *  - Errors: arguments are checked on the host before anything is launched;
  *    a bad argument returns AB_ERR_INVALID_ARG (or AB_ERR_UNSUPPORTED for a
  *    valid but unimplemented size) and enqueues nothing.  AB_ERR_CUDA reports
@@ -262,8 +262,9 @@ ab_status ab_forward_slice(const ab_params* p, int32_t bh0, int32_t nbh, const v
  * heads (every (b, h) is independent): the inputs of one group cross PCIe on
  * an internal stream while the previous group computes on `stream` and the
  * one before it copies back on a second internal stream; the two streams and
- * their events are created by the call and released when its work completes,
- * and `stream` waits for all of it.  Otherwise everything is enqueued on
+ * their events are created on the context's first pipelined call and reused
+ * (calls from several host threads take turns enqueueing), and `stream`
+ * waits for all of it.  Otherwise everything is enqueued on
  * `stream`.  O_host is valid once `stream` has been synchronised.  The device
  * buffers are owned by the caller.
  */
