@@ -97,11 +97,12 @@ def peaks():
 
 # DRAM traffic of one sparse attention launch, from the ncu capture of the
 # 8-head case of the Wan2.1-480p layer (dram__bytes_read.sum +
-# dram__bytes_write.sum = 205.877 MB + 51.283 MB, kv_block 16, 11 % kept),
-# scaled to the layer's heads (the launch's traffic grows with the heads).  It
-# describes the kernel sources it was measured on only: with any other
-# sources (hash below) the bench reports null.
-ATTN_TRAFFIC = {"sources_sha256_16": "cd33bbc67a456aa8", "bytes_per_head": (205.955328e6 + 52.344832e6) / 8,
+# dram__bytes_write.sum = 206.222 MB + 53.658 MB, kv_block 16, 11 % kept;
+# summarised under profiles/), scaled to the layer's heads (the launch's
+# traffic grows with the heads).  It describes the kernel sources it
+# was measured on only: with any other sources (hash below) the bench reports
+# null.
+ATTN_TRAFFIC = {"sources_sha256_16": "91ae4471fe2799dc", "bytes_per_head": (206.221568e6 + 53.658368e6) / 8,
                 "workload": "wan480", "kv_block": 16, "keep_ratio": 0.11}
 
 
