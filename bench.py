@@ -296,6 +296,25 @@ def tile_flop(w, cnt) -> float:
     return 4.0 * 128 * 128 * w.d * float(tiles.sum())
 
 
+# Bytes one SM's TMA unit brings into shared memory per clock at most: a
+# probe issuing back-to-back 32 KB tile loads into one SM (any grid size)
+# measured 32 B per clock (about 48 cycles per box + 32 B per clock; 30 B at
+# 16 KB boxes, 23 B at 4 KB boxes issued one at a time).
+TMA_INGRESS_B_PER_CLK_SM = 32.0
+NUM_SMS = 148
+
+
+def ingress_bytes(w, cnt) -> float:
+    """Bytes the sparse attention kernel brings into shared memory per
+    launch: the two query blocks' Q tiles of every CTA and, per tile of
+    128 keys, one K and one V tile (128 rows x d bf16 each, list padding
+    included)."""
+    slots = 128 // w.kv_block
+    tiles = (np.asarray(cnt, np.int64) + slots - 1) // slots
+    tile_bytes = 128 * w.d * 2
+    return float(tiles.sum()) * 2 * tile_bytes + w.B * w.H * w.Nq * tile_bytes
+
+
 def whole_job_value(w, world: int, ms_step: float) -> float:
     """Dense-equivalent TFLOP/s of the whole job: every rank processes one layer per step."""
     return dense_flop(w) * world / (ms_step * 1e-3) / 1e12
@@ -415,6 +434,7 @@ def run_ours(args):
                          "traffic_note": "ncu dram bytes of the 8-head capture x H/8 (profiles/)",
                          "kernel": "ab_attention_kernel<128,16>", "peak_kind": peak_kind,
                          "per_launch_flop": exec_flop},
+            "ingress": ingress_roofline(w, cnt, att_avg, clk),
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk,
@@ -608,6 +628,20 @@ def quality(ab, p, Q, K, V, bufs, dev):
             "ms_sample_systematic": round(t2.elapsed_time(t3) / 3, 4),
             "ms_sample_truncation": round(t0.elapsed_time(t1) / 3, 4),
             "note": "same P and budget; information only, not a gate"}
+
+
+def ingress_roofline(w, cnt, att_ms, clk):
+    """Second roofline of the attention kernel: bytes its TMA loads bring into
+    each SM's shared memory per SM clock (the median SM clock sampled during
+    the timed region) against the probe's 32 B per clock."""
+    mhz = clk.get("sm_mhz") if isinstance(clk, dict) else None
+    b = ingress_bytes(w, cnt)
+    if not mhz:
+        return {"bytes_per_launch": b, "achieved": None, "note": "no SM clock sample"}
+    per_clk = b / (att_ms * 1e-3 * mhz * 1e6 * NUM_SMS)
+    return {"bound": "tma_ingress", "achieved": round(per_clk, 2), "peak": TMA_INGRESS_B_PER_CLK_SM,
+            "unit": "B/clk per SM", "frac": round(per_clk / TMA_INGRESS_B_PER_CLK_SM, 4), "bytes_per_launch": b,
+            "sm_mhz": mhz, "peak_kind": "probe (TMA tile loads into one SM, not driver-measured)"}
 
 
 def time_fused_select_sample(ab, p, Q, K, dev, iters=3):
