@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -199,7 +200,7 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, floa
     if (sip) a.sip = *sip;
     const int G = 128 / d.C;
     const unsigned grid = unsigned(d.BH * ((d.Nq + G - 1) / G));
-    const int smem = ScSmem<D>::kAlloc;
+    const int smem = sip ? ScSmem<D, true>::kAlloc : ScSmem<D>::kAlloc;
     auto launch = [&](auto kern) -> ab_status {
       if (set_smem(kern, smem) != cudaSuccess) return AB_ERR_CUDA;
       kern<<<grid, 288, smem, st>>>(tmCent, tmKsum, a);
@@ -287,6 +288,23 @@ ab_status do_select(const Dims& d, const void* Q, const void* K, float* P, float
 
 // rows: the rows of this call (d.BH * d.Nq unless a caller processes a range of
 // heads); H and row0 place them in the full problem for the draws' counters.
+// One warp per row (the row's quantised weights in shared memory), for rows
+// of at most 2048 blocks: the smallest chunk count that holds the row.
+template <bool kSystematic>
+ab_status launch_sip_warp(const SipArgs& a, int rows, int Nkv, cudaStream_t st) {
+  auto go = [&](auto kmax) -> ab_status {
+    constexpr int KMAX = decltype(kmax)::value;
+    constexpr int smem = 8 * 32 * KMAX * 16;
+    if (smem > 48 * 1024 && set_smem(sip_warp_kernel<KMAX, kSystematic>, smem) != cudaSuccess)
+      return AB_ERR_CUDA;
+    sip_warp_kernel<KMAX, kSystematic><<<unsigned((rows + 7) / 8), 256, smem, st>>>(a, rows);
+    return launch_status();
+  };
+  if (Nkv <= 512) return go(std::integral_constant<int, 4>{});
+  if (Nkv <= 1024) return go(std::integral_constant<int, 8>{});
+  return go(std::integral_constant<int, 16>{});
+}
+
 ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count, cudaStream_t st,
                     int H = -1, int64_t row0 = 0) {
   if (!P || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
@@ -297,8 +315,8 @@ ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q3
   a.seed_lo = uint32_t(d.seed); a.seed_hi = uint32_t(d.seed >> 32);
   a.row0 = row0;
   const int rows = d.BH * d.Nq;
-  if (d.Nkv <= 2048) {  // one warp per row, the row in registers
-    sip_warp_kernel<16, false><<<unsigned((rows + 7) / 8), 256, 0, st>>>(a, rows);
+  if (d.Nkv <= 2048) {  // one warp per row
+    return launch_sip_warp<false>(a, rows, d.Nkv, st);
   } else if (d.Nkv <= kSipSmemCap) {
     const int smem = 16 * ((d.Nkv + 3) / 4);
     if (smem > 48 * 1024 &&
@@ -460,8 +478,8 @@ ab_status ab_sample_systematic(const ab_params* p, const float* P, int32_t* idx,
   a.seed_lo = uint32_t(d.seed); a.seed_hi = uint32_t(d.seed >> 32);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int rows = d.BH * d.Nq;
-  if (d.Nkv <= 2048) {  // one warp per row, the row in registers
-    sip_warp_kernel<16, true><<<unsigned((rows + 7) / 8), 256, 0, st>>>(a, rows);
+  if (d.Nkv <= 2048) {  // one warp per row
+    return launch_sip_warp<true>(a, rows, d.Nkv, st);
   } else if (d.Nkv <= kSipSmemCap) {
     const int smem = 16 * ((d.Nkv + 3) / 4);
     if (smem > 48 * 1024 &&

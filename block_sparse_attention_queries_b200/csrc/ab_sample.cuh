@@ -334,19 +334,23 @@ __global__ void __launch_bounds__(kSipThreads) sip_kernel(const SipArgs a) {
 
 // One warp per row, for rows of at most 32 * 4 * KMAX blocks: the same
 // arithmetic as sip_kernel (results are identical integers), with the
-// quantised row in registers and warp shuffles instead of block barriers.
+// quantised row in the warp's own slice of shared memory and warp shuffles
+// instead of block barriers.
 // Lane l owns blocks j = 128 k + 4 l + q (k < KMAX, q < 4), i.e. the same 4
 // consecutive blocks per Philox call.  kSystematic: systematic sampling with
 // the same Pi (as systematic_pass: one offset U per row, block j kept iff a
 // point U + m 2^32 lies in [C_j, C_j + Pi_j), C_j the running sum of Pi in
 // ascending j, here a warp scan per 128-block chunk).
 // One warp samples row `row` of a.P (Nkv <= 128 KMAX), the whole row's
-// quantised weights in registers (KMAX x 4 per lane).  kCoherent: P was
-// written earlier by the calling kernel itself, so it is read through L2
-// (__ldcg) rather than the read-only path, which is only valid for data the
-// kernel does not write.
+// quantised weights in this warp's KMAX x 512 bytes of shared memory at
+// `wsm` (16-byte aligned; lane l keeps its four weights of chunk k at uint4
+// index 32 k + l, so a warp's loads are contiguous).  Holding the row in
+// registers instead (64 per lane at KMAX = 16) left 16 warps per SM and
+// took 9 % longer.  kCoherent: P was written earlier by the calling kernel
+// itself, so it is read through L2 (__ldcg) rather than the read-only path,
+// which is only valid for data the kernel does not write.
 template <int KMAX, bool kSystematic, bool kCoherent>
-__device__ __forceinline__ void sip_warp_row(const SipArgs& a, int row) {
+__device__ __forceinline__ void sip_warp_row(const SipArgs& a, int row, uint4* wsm) {
   static_assert(KMAX * 4 * 16777216ull < 4294967296ull, "per-lane partial sums must fit 32 bits");
   const int lane = threadIdx.x & 31;
   auto loadP = [](const float* p) { return kCoherent ? __ldcg(p) : __ldg(p); };
@@ -356,14 +360,17 @@ __device__ __forceinline__ void sip_warp_row(const SipArgs& a, int row) {
   const int i = int(grow % a.Nq);
   const int Nkv = a.Nkv;
   const float* P = a.P + int64_t(row) * Nkv;
-  uint32_t w[KMAX][4];
+  // the four weights of chunk k of this lane
+  auto wk = [&](int k) -> uint4 { return wsm[32 * k + lane]; };
 #pragma unroll
   for (int k = 0; k < KMAX; ++k) {
+    uint32_t v[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int j = 128 * k + 4 * lane + q;
-      w[k][q] = j < Nkv ? quantise_w(loadP(P + j)) : 0u;  // entries >= Nkv: 0, never capped
+      v[q] = j < Nkv ? quantise_w(loadP(P + j)) : 0u;  // entries >= Nkv: 0, never capped
     }
+    wsm[32 * k + lane] = make_uint4(v[0], v[1], v[2], v[3]);
   }
 
   // ---- capping threshold (fixed point)
@@ -373,11 +380,13 @@ __device__ __forceinline__ void sip_warp_row(const SipArgs& a, int row) {
     uint32_t ncap = 0, part = 0;
 #pragma unroll
     for (int k = 0; k < KMAX; ++k) {
+      const uint4 v4 = wk(k);
+      const uint32_t v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const bool cap = w[k][q] >= theta;
+        const bool cap = v[q] >= theta;
         ncap += cap ? 1u : 0u;
-        part += cap ? 0u : w[k][q];
+        part += cap ? 0u : v[q];
       }
     }
     uint64_t sum = part;
@@ -413,12 +422,14 @@ __device__ __forceinline__ void sip_warp_row(const SipArgs& a, int row) {
     for (int k = 0; k < KMAX; ++k) {
       if (128 * k >= Nkv) break;  // warp-uniform
       const int j0 = 128 * k + 4 * lane;
+      const uint4 v4 = wk(k);
+      const uint32_t v[4] = {v4.x, v4.y, v4.z, v4.w};
       uint64_t pis[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         pis[q] = j0 + q >= Nkv ? 0ull
-                 : w[k][q] >= theta ? (1ull << 32)
-                                    : uint64_t(pi_free(uint64_t(R32) * w[k][q], S_hi, S_lo, inv_s32));
+                 : v[q] >= theta ? (1ull << 32)
+                                 : uint64_t(pi_free(uint64_t(R32) * v[q], S_hi, S_lo, inv_s32));
       const uint64_t mine = (pis[0] + pis[1]) + (pis[2] + pis[3]);
       uint64_t incl = mine;
 #pragma unroll
@@ -464,13 +475,15 @@ __device__ __forceinline__ void sip_warp_row(const SipArgs& a, int row) {
         const uint4 u4 = philox4x32_10(make_uint4(uint32_t(j0 >> 2), uint32_t(i), uint32_t(h), uint32_t(b)),
                                        a.seed_lo, a.seed_hi);
         const uint32_t us[4] = {u4.x, u4.y, u4.z, u4.w};
+        const uint4 v4 = wk(k);
+        const uint32_t v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           bool keep;
-          if (w[k][q] >= theta) {
+          if (v[q] >= theta) {
             keep = true;
           } else {
-            const uint64_t X = uint64_t(R32) * w[k][q];
+            const uint64_t X = uint64_t(R32) * v[q];
             keep = us[q] == 0u || mul_le_shift32(us[q], S_hi, S_lo, X);
           }
           if (keep && j0 + q < Nkv) keep_mask |= 1u << q;
@@ -501,12 +514,15 @@ __device__ __forceinline__ void sip_warp_row(const SipArgs& a, int row) {
   }
 }
 
-// One warp per row for rows of at most 128 KMAX blocks.
+// One warp per row for rows of at most 128 KMAX blocks, 8 warps per CTA,
+// each with its row in KMAX x 512 bytes of dynamic shared memory.
 template <int KMAX, bool kSystematic>
-__global__ void __launch_bounds__(256) sip_warp_kernel(const SipArgs a, int rows) {
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+__global__ void __launch_bounds__(256, 3) sip_warp_kernel(const SipArgs a, int rows) {
+  extern __shared__ uint4 sip_rows[];  // [8 warps][32 KMAX]
+  const int warp = threadIdx.x >> 5;
+  const int row = blockIdx.x * 8 + warp;
   if (row >= rows) return;  // whole warp: no block-level synchronisation below
-  sip_warp_row<KMAX, kSystematic, false>(a, row);
+  sip_warp_row<KMAX, kSystematic, false>(a, row, sip_rows + warp * 32 * KMAX);
 }
 
 // Truncation, the selection SIP is contrasted with (AB-Attention page,

@@ -335,19 +335,22 @@ __device__ __forceinline__ float max_tree(const float* v) {
 }
 
 // ------------------------------------------------------------------ scores
-template <int D>
+template <int D, bool kSample = false>
 struct ScSmem {
   static constexpr int kSlabs = D / 64;
+  static constexpr int kSampleRows = 9 * 16 * 512;  // kSample: nine warps' quantised rows, over A and B
   static constexpr int kA = kSlabs * 16384;          // 128 centroid rows x D bf16
   static constexpr int kB = kSlabs * 16384;          // 128 K summaries x D bf16 (one chunk)
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kA;           // 2 stages
-  static constexpr int kOffW = kOffB + 2 * kB;       // float [128] row weights
+  static constexpr int kEndB = kOffB + 2 * kB;
+  static constexpr int kOffW = kSample && kSampleRows > kEndB ? kSampleRows : kEndB;  // float [128] row weights
   static constexpr int kOffX = kOffW + 512;          // float [2 halves][2][128] max/sum exchange
   static constexpr int kOffBar = kOffX + 2048;       // a_full, b_full[2], b_empty[2], s_full[2], t_free[2], drain, xch
   static constexpr int kOffMisc = kOffBar + 12 * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
+  static_assert(!kSample || kSampleRows <= kOffW, "the sampling rows end before the row weights");
 };
 
 struct ScoreArgs {
@@ -384,7 +387,8 @@ __device__ __forceinline__ void group_reduce_scatter(float (&v)[32], int lane) {
 // MMAs.  Two CTAs share an SM (96 KB of shared memory, 256 TMEM columns each).  The two column halves of a row keep separate running max / sum in
 // the first pass and merge them before the second.
 // kSample (rows of at most 2048 blocks): once the CTA's rows of P are written,
-// its nine warps run SIP on them (sip_warp_row, one warp per row), so the
+// its nine warps run SIP on them (sip_warp_row, one warp per row, each row's
+// weights in 8 KB of the shared memory the scoring no longer uses), so the
 // sampling of these rows starts as soon as their estimate exists, next to the
 // scoring of the other CTAs, without a second launch or a DRAM round trip of
 // P (it is read back from L2).
@@ -392,7 +396,7 @@ template <int D, int C, bool kSample = false>
 __global__ void __launch_bounds__(288, 2)
     score_kernel(const __grid_constant__ CUtensorMap tmCent, const __grid_constant__ CUtensorMap tmKsum,
                  const ScoreArgs a) {
-  using SM = ScSmem<D>;
+  using SM = ScSmem<D, kSample>;
   constexpr int G = 128 / C;  // query blocks per CTA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -580,7 +584,7 @@ __global__ void __launch_bounds__(288, 2)
     if (!*abort_flag) {
       for (int r = warp; r < G; r += 9) {
         const int i = i0 + r;
-        if (i < a.Nq) sip_warp_row<16, false, true>(a.sip, bh * a.Nq + i);
+        if (i < a.Nq) sip_warp_row<16, false, true>(a.sip, bh * a.Nq + i, reinterpret_cast<uint4*>(smem) + warp * 32 * 16);
       }
     }
   }
