@@ -412,6 +412,7 @@ def run_ours(args):
             dense_ms = run_dense(ab, p, Q, K, V, dev, 3)
             qual = quality(ab, p, Q, K, V, bufs, dev)
             qual["ms_select_sample_fused"] = time_fused_select_sample(ab, p, Q, K, dev)
+            qual.update(mass_found(w, Q, K, bufs.P, ab.budget(p)))
             qual["concentrated"] = quality_concentrated(ab, w, dev)
             cpu = cpu_baseline(w, args, Qc, Kc, Vc)
         out = {
@@ -661,6 +662,30 @@ def time_fused_select_sample(ab, p, Q, K, dev, iters=3):
     return round(t0.elapsed_time(t1) / iters, 4)
 
 
+def mass_found(w, Q, K, P, Kb, heads=(0, 1, 2, 3), blocks=4):
+    """Information only: on sampled query blocks, the share of the block's
+    attention mass (dense softmax of its queries, averaged over its rows,
+    summed per KV block) held by the Kb blocks with the largest P (what the
+    IBCS estimate finds) and by the Kb blocks with the largest true mass (the
+    ideal top-Kb).  A diagnostic computed with plain torch ops on the GPU,
+    outside the timed path."""
+    import math
+    import torch
+    found, ideal = [], []
+    for h in heads:
+        for i in sorted({int(round(k * (w.Nq - 1) / max(1, blocks - 1))) for k in range(blocks)}):
+            q = Q[0, h, i * w.q_block:(i + 1) * w.q_block].float()
+            logits = (q @ K[0, h].float().T) / math.sqrt(w.d)
+            prob = torch.softmax(logits, dim=-1).mean(0)                       # [Lk]
+            pad = w.Nkv * w.kv_block - prob.numel()
+            mass = torch.nn.functional.pad(prob, (0, pad)).view(w.Nkv, w.kv_block).sum(1).double()
+            sel = torch.topk(P[0, h, i].double(), Kb).indices
+            found.append(float(mass[sel].sum()))
+            ideal.append(float(torch.topk(mass, Kb).values.sum()))
+    return {"mass_found_by_P_topKb": round(sum(found) / len(found), 4),
+            "mass_ideal_topKb": round(sum(ideal) / len(ideal), 4), "query_blocks_sampled": len(found)}
+
+
 def quality_concentrated(ab, w, dev, heads=8, s_peak=32.0):
     """Information only: the relative L2 distance to dense attention of SIP,
     systematic sampling and truncation at the same budget when attention is
@@ -683,9 +708,11 @@ def quality_concentrated(ab, w, dev, heads=8, s_peak=32.0):
     def rel(o):
         return round(float(torch.linalg.vector_norm(o.double() - Od.double()) / ref), 5)
 
-    return {"s_peak": s_peak, "heads": wc.H, "rel_l2_sip_vs_dense": rel(b.O),
-            "rel_l2_systematic_vs_dense": rel(Os), "rel_l2_truncation_vs_dense": rel(Ot),
-            "kept_block_fraction": round(float(b.count.sum()) / (wc.B * wc.H * wc.Nq * wc.Nkv), 5)}
+    out = {"s_peak": s_peak, "heads": wc.H, "rel_l2_sip_vs_dense": rel(b.O),
+           "rel_l2_systematic_vs_dense": rel(Os), "rel_l2_truncation_vs_dense": rel(Ot),
+           "kept_block_fraction": round(float(b.count.sum()) / (wc.B * wc.H * wc.Nq * wc.Nkv), 5)}
+    out.update(mass_found(wc, Q, K, b.P, ab.budget(p)))
+    return out
 
 
 # ---------------------------------------------------------- CPU oracle arm
