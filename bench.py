@@ -693,10 +693,13 @@ def quality_concentrated(ab, w, dev, heads=8, s_peak=32.0):
     sqrt(d) of two tokens at the same position is about 32: a few blocks hold
     most of each row's weight), on the first `heads` heads of the workload."""
     import torch
-    from block_sparse_attention_queries_b200.synthetic import make_qkv
+    from block_sparse_attention_queries_b200.synthetic import make_cross_qkv, make_qkv
     wc = w.with_(H=min(heads, w.H))
     p = ab.Params.of(wc, seed=42)
-    Qc, Kc, Vc = make_qkv(wc.B, wc.H, wc.grid, wc.d, wc.F, s_peak=s_peak)
+    if wc.grid_kv is not None:
+        Qc, Kc, Vc = make_cross_qkv(wc.B, wc.H, wc.grid, wc.grid_kv, wc.d, wc.F, s_peak=s_peak)
+    else:
+        Qc, Kc, Vc = make_qkv(wc.B, wc.H, wc.grid, wc.d, wc.F, s_peak=s_peak)
     Q, K, V = (t.to(dev) for t in (Qc, Kc, Vc))
     b = ab.ab_forward(p, Q, K, V)
     Od = ab.ab_attention_dense(p, Q, K, V)

@@ -468,6 +468,50 @@ def test_forward_host_equals_device_path(dev, B, H, grid):
     assert torch.equal(Oh, ref.O.cpu())
 
 
+def test_forward_host_repeated_and_from_two_threads(dev):
+    # the pipelined host call keeps its copy streams and events per CUDA
+    # context: repeated calls, and calls from two host threads at once (each
+    # on its own stream with its own buffers), all give ab_forward's results
+    import threading
+    grid = (2, 16, 16)
+    p = ab.Params(B=1, H=9, L=512, d=128, q_block=128, kv_block=16, C=8, keep_ratio=0.15, seed=5)
+    (Qc, Kc, Vc), (Q, K, V), _ = _inputs(p, grid, 8, 21, dev)
+    ref = ab.ab_forward(p, Q, K, V)
+    torch.cuda.synchronize()
+    results, errors = {}, []
+
+    def worker(k):
+        try:
+            st = torch.cuda.Stream(dev)
+            with torch.cuda.stream(st):
+                Qh, Kh, Vh = (t.pin_memory() for t in (Qc, Kc, Vc))
+                Oh = torch.empty_like(Qc).pin_memory()
+                Qd, Kd, Vd = (torch.empty_like(t) for t in (Q, K, V))
+                bufs = ab.Buffers(p, dev)
+                Oh.zero_()
+                for _ in range(3):
+                    ab.ab_forward_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, bufs, dev)
+                st.synchronize()
+                res = (Oh.clone(), bufs.idx.clone(), bufs.count.clone())
+                st.synchronize()
+                results[k] = res
+        except Exception as e:  # reported below, on the main thread
+            errors.append(repr(e))
+
+    threads = [threading.Thread(target=worker, args=(k,)) for k in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    _no_device_error(dev)
+    for k in range(2):
+        Oh, idx, cnt = results[k]
+        assert torch.equal(cnt, ref.count)
+        assert torch.equal(idx, ref.idx)
+        assert torch.equal(Oh, ref.O.cpu())
+
+
 @pytest.mark.parametrize("d,kvb", [(128, 16), (64, 32), (128, 64)])
 def test_full_budget_equals_dense_bitwise(dev, d, kvb):
     grid = (4, 18, 20)  # L = 1440: ragged last query block and last KV block for 64
