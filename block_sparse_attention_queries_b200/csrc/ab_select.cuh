@@ -72,11 +72,13 @@ __global__ void __launch_bounds__(256) ksum_kernel(const __nv_bfloat16* __restri
 }
 
 // ----------------------------------------------------------------- k-means
-// Shared memory of one k-means CTA.  The one-hot assignment tile aliases the
-// lo-part centroid tile: the distance product that reads the lo part has
-// completed before the one-hot is written, and the sum product that reads
-// the one-hot has completed before the next lo part is written.  Rows >= C of
-// both stay zero.
+// Shared memory of one k-means CTA.  With C <= 8 the hi tile holds the hi
+// parts in rows 0 .. C-1 and the lo parts in rows C .. 2C-1, and the second
+// tile is the one-hot assignment tile alone; with C = 16 the one-hot tile
+// aliases the lo-part tile: the distance product that reads the lo part has
+// completed before the one-hot is written, and the sum product that reads the
+// one-hot has completed before the next lo part is written.  Rows no part or
+// cluster uses stay zero.
 template <int D>
 struct KmSmem {
   static constexpr int kOffQ = 0;                      // 128 x 128 bf16, SW128 slabs of 16 KB (slab 1 unused if D = 64)
@@ -126,8 +128,11 @@ __device__ __forceinline__ float warp_sum_scatter(const float (&in)[N]) {
 // One CTA (128 threads) per query block.  Thread e < D keeps dimension e of
 // every centroid in registers.  Per Lloyd iteration, two small tensor-core
 // products:
-//   distances  q . mu_c = Q (128 x d) x [mu_hi; mu_lo]^T (d x 16), thread q
-//              reads its 16 columns and takes argmin |mu_c|^2 - 2 q . mu_c;
+//   distances  q . mu_c = Q (128 x d) x [mu_hi; mu_lo]^T: for C <= 8 one
+//              product with N = 16 (hi parts in columns c, lo parts in C + c,
+//              added by the thread; half the MMAs to issue), for C = 16 two
+//              products accumulating in the same 16 columns; thread q reads
+//              its columns and takes argmin |mu_c|^2 - 2 q . mu_c;
 //   sums       sum_{q in c} q = Q^T (d x 128) x onehot (128 x 16): Q is read
 //              as an MN-major operand (d contiguous), so thread e receives the
 //              sums of dimension e for every cluster in 16 TMEM columns.
@@ -194,6 +199,15 @@ __global__ void __launch_bounds__(128, C <= 8 ? 5 : 3) kmeans_kernel(const __gri
 
   const uint32_t id_dist = idesc_bf16_f32(128, 16, 0, 0);  // Q (K-major) x mu parts (K-major)
   const uint32_t id_sum = idesc_bf16_f32(128, 16, 1, 0);   // Q^T (MN-major) x onehot (K-major)
+  // With C <= 8 the lo parts sit in rows C .. 2C-1 of the hi tile, so one
+  // N = 16 product gives both (columns c and C + c); with C = 16 they take
+  // a tile and a product of their own.
+  constexpr bool kPacked = 2 * C <= 16;
+  // operand descriptors, built once; each MMA adds its byte offset
+  const SmemDesc dq = smem_desc_base(sbase + SM::kOffQ, 16, 1024);        // Q, K-major
+  const SmemDesc dqt = smem_desc_base(sbase + SM::kOffQ, 16384, 1024);    // Q read MN-major
+  const SmemDesc dhi = smem_desc_base(sbase + SM::kOffBhi, 16, 1024);
+  const SmemDesc dlo = smem_desc_base(sbase + SM::kOffBlo, 16, 1024);     // lo parts / one-hot
   uint32_t phase = 0;
   for (int it = 0; it < iters && ok; ++it) {
     // centroid tiles: bf16 hi and lo parts of mu (row c, column e); partial |mu_c|^2
@@ -204,9 +218,12 @@ __global__ void __launch_bounds__(128, C <= 8 ? 5 : 3) kmeans_kernel(const __gri
       if (own_dim) {
         const __nv_bfloat16 hi = __float2bfloat16_rn(mu[c]);
         const __nv_bfloat16 lo = __float2bfloat16_rn(mu[c] - __bfloat162float(hi));
-        const uint32_t off = sw_tile_off(2048, c, tid);
-        *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffBhi + off) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffBlo + off) = lo;
+        *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffBhi + sw_tile_off(2048, c, tid)) = hi;
+        if constexpr (kPacked) {
+          *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffBhi + sw_tile_off(2048, C + c, tid)) = lo;
+        } else {
+          *reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffBlo + sw_tile_off(2048, c, tid)) = lo;
+        }
       }
     }
     {
@@ -223,10 +240,8 @@ __global__ void __launch_bounds__(128, C <= 8 ? 5 : 3) kmeans_kernel(const __gri
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
         const uint32_t boff = (kk >> 2) * 2048 + (kk & 3) * 32;
-        mma_bf16_ss(tmem, smem_desc_sw128(sbase + SM::kOffQ + aoff, 16, 1024),
-                    smem_desc_sw128(sbase + SM::kOffBhi + boff, 16, 1024), id_dist, kk > 0 ? 1u : 0u);
-        mma_bf16_ss(tmem, smem_desc_sw128(sbase + SM::kOffQ + aoff, 16, 1024),
-                    smem_desc_sw128(sbase + SM::kOffBlo + boff, 16, 1024), id_dist, 1u);
+        mma_bf16_ss(tmem, desc_at(dq, aoff), desc_at(dhi, boff), id_dist, kk > 0 ? 1u : 0u);
+        if constexpr (!kPacked) mma_bf16_ss(tmem, desc_at(dq, aoff), desc_at(dlo, boff), id_dist, 1u);
       }
       mma_commit(bar_mma);
     }
@@ -247,7 +262,8 @@ __global__ void __launch_bounds__(128, C <= 8 ? 5 : 3) kmeans_kernel(const __gri
       for (int c = 0; c < C; ++c) {
         const float4 p4 = *reinterpret_cast<const float4*>(musq_part + 4 * c);
         const float musq = (p4.x + p4.y) + (p4.z + p4.w);
-        const float dist = fmaf(-2.f, __uint_as_float(dv[c]), musq);
+        const float dot = kPacked ? __uint_as_float(dv[c]) + __uint_as_float(dv[C + c]) : __uint_as_float(dv[c]);
+        const float dist = fmaf(-2.f, dot, musq);
         if (dist < bd) {  // strict: ties go to the lower c
           bd = dist;
           best = c;
@@ -270,8 +286,7 @@ __global__ void __launch_bounds__(128, C <= 8 ? 5 : 3) kmeans_kernel(const __gri
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)  // K = 128 queries, 16 per step
-        mma_bf16_ss(tmem + 16u, smem_desc_sw128(sbase + SM::kOffQ + kk * 2048, 16384, 1024),
-                    smem_desc_sw128(sbase + SM::kOffBlo + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), id_sum,
+        mma_bf16_ss(tmem + 16u, desc_at(dqt, kk * 2048), desc_at(dlo, (kk >> 2) * 2048 + (kk & 3) * 32), id_sum,
                     kk > 0 ? 1u : 0u);
       mma_commit(bar_mma);
     }
