@@ -286,8 +286,6 @@ ab_status do_select(const Dims& d, const void* Q, const void* K, float* P, float
   return d.d == 128 ? run_select<128>(d, Q, K, P, cent, counts, w, st) : run_select<64>(d, Q, K, P, cent, counts, w, st);
 }
 
-// rows: the rows of this call (d.BH * d.Nq unless a caller processes a range of
-// heads); H and row0 place them in the full problem for the draws' counters.
 // One warp per row (the row's quantised weights in shared memory), for rows
 // of at most 2048 blocks: the smallest chunk count that holds the row.
 template <bool kSystematic>
@@ -305,6 +303,8 @@ ab_status launch_sip_warp(const SipArgs& a, int rows, int Nkv, cudaStream_t st) 
   return go(std::integral_constant<int, 16>{});
 }
 
+// rows: the rows of this call (d.BH * d.Nq unless a caller processes a range of
+// heads); H and row0 place them in the full problem for the draws' counters.
 ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count, cudaStream_t st,
                     int H = -1, int64_t row0 = 0) {
   if (!P || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
@@ -329,7 +329,7 @@ ab_status do_sample(const Dims& d, const float* P, int32_t* idx, uint32_t* pi_q3
   return launch_status();
 }
 
-constexpr int kFusedSampleMaxNkv = 2048;  // rows the scoring kernel's warps sample in registers
+constexpr int kFusedSampleMaxNkv = 2048;  // rows the scoring kernel's warps sample (8 KB of shared memory each)
 
 // ab_select then ab_sample; for rows of at most kFusedSampleMaxNkv blocks in
 // one launch less (the scoring kernel samples the rows it has just scored).
