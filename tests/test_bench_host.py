@@ -61,3 +61,20 @@ def test_tile_flop_counts_full_tiles():
     for r in np.ndindex(*c.shape):
         idx[r][:c[r]] = np.sort(rng.choice(w.Nkv, c[r], replace=False))
     assert bench.tile_flop(w, c) >= bench.executed_flop(w, c, idx)
+
+
+def test_ingress_bytes_and_roofline():
+    # per CTA two Q tiles; per 128-key tile of a list one K and one V tile of
+    # 128 x d bf16 (padding of the last tile included)
+    w = WORKLOADS["wan480"].with_(H=1)
+    tile = 128 * w.d * 2
+    cnt = np.zeros((1, 1, w.Nq), np.int64)
+    cnt[0, 0, :3] = [1, 8, 9]  # 1, 1 and 2 tiles of 8 blocks
+    assert bench.ingress_bytes(w, cnt) == (1 + 1 + 2) * 2 * tile + w.Nq * tile
+    w32 = w.with_(kv_block=32)  # 4 blocks per tile
+    assert bench.ingress_bytes(w32, cnt) == (1 + 2 + 3) * 2 * tile + w.Nq * tile
+    r = bench.ingress_roofline(w, cnt, 1.0, {"sm_mhz": 1000.0})
+    expect = bench.ingress_bytes(w, cnt) / (1e-3 * 1e9 * bench.NUM_SMS)
+    assert abs(r["achieved"] - round(expect, 2)) < 1e-9
+    assert r["frac"] == round(expect / bench.TMA_INGRESS_B_PER_CLK_SM, 4)
+    assert bench.ingress_roofline(w, cnt, 1.0, {"error": "no samples"})["achieved"] is None
