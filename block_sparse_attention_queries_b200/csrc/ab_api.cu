@@ -337,14 +337,15 @@ constexpr int kFusedSampleMaxNkv = 2048;  // rows the scoring kernel's warps sam
 ab_status do_select_sample(const Dims& d, const void* Q, const void* K, float* P, int32_t* idx, uint32_t* pi_q32,
                            int32_t* count, void* ws, size_t ws_bytes, cudaStream_t st, int H = -1,
                            int64_t row0 = 0) {
-  if (d.Nkv > kFusedSampleMaxNkv) {
-    const ab_status s = do_select(d, Q, K, P, nullptr, nullptr, ws, ws_bytes, st);
-    return s != AB_OK ? s : do_sample(d, P, idx, pi_q32, count, st, H, row0);
-  }
+  // every argument is checked before anything is enqueued, on both paths
   if (!Q || !K || !P || !ws || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(P) || !aligned16(ws)) return AB_ERR_INVALID_ARG;
   if (!aligned16(idx) || !aligned16(pi_q32) || !aligned16(count)) return AB_ERR_INVALID_ARG;
   if (ws_bytes < workspace_layout(d).total) return AB_ERR_WORKSPACE;
+  if (d.Nkv > kFusedSampleMaxNkv) {
+    const ab_status s = do_select(d, Q, K, P, nullptr, nullptr, ws, ws_bytes, st);
+    return s != AB_OK ? s : do_sample(d, P, idx, pi_q32, count, st, H, row0);
+  }
   SipArgs a{};
   a.P = P; a.idx = idx; a.pi_q32 = pi_q32; a.count = count;
   a.H = H > 0 ? H : d.H; a.Nq = d.Nq; a.Nkv = d.Nkv; a.Kb = d.Kb;
@@ -353,6 +354,18 @@ ab_status do_select_sample(const Dims& d, const void* Q, const void* K, float* P
   auto* w = reinterpret_cast<uint8_t*>(ws);
   return d.d == 128 ? run_select<128>(d, Q, K, P, nullptr, nullptr, w, st, &a)
                     : run_select<64>(d, Q, K, P, nullptr, nullptr, w, st, &a);
+}
+
+// Every device argument of a whole-path call (select, sample, attention),
+// checked before anything is enqueued: non-null, 16-byte aligned, and a
+// workspace of at least ws_need bytes.
+ab_status check_path_args(const void* Q, const void* K, const void* V, const float* P, const int32_t* idx,
+                          const uint32_t* pi_q32, const int32_t* count, const void* O, const void* ws,
+                          size_t ws_bytes, size_t ws_need) {
+  const void* ptrs[] = {Q, K, V, P, idx, pi_q32, count, O, ws};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return AB_ERR_INVALID_ARG;
+  return ws_bytes < ws_need ? AB_ERR_WORKSPACE : AB_OK;
 }
 
 ab_status do_attention(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* idx,
@@ -531,7 +544,8 @@ ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const voi
   NvtxRange nvtx("ab_forward");
   ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
-  if (!V || !O || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
+  s = check_path_args(Q, K, V, P, idx, pi_q32, count, O, workspace, ws_bytes, workspace_layout(d).total);
+  if (s != AB_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   s = do_select(d, Q, K, P, nullptr, nullptr, workspace, ws_bytes, st);
   if (s != AB_OK) return s;
@@ -548,12 +562,13 @@ ab_status ab_forward_slice(const ab_params* p, int32_t bh0, int32_t nbh, const v
   ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
   if (nbh < 1 || bh0 < 0 || int64_t(bh0) + nbh > int64_t(d.BH)) return AB_ERR_INVALID_ARG;
-  if (!V || !O || !idx || !pi_q32 || !count) return AB_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the slice as a problem of its own (B = 1, H = nbh); the draws keep the
   // whole problem's counters (its H and the slice's first row)
   Dims dc = d;
   dc.B = 1; dc.H = nbh; dc.BH = nbh;
+  s = check_path_args(Q, K, V, P, idx, pi_q32, count, O, workspace, ws_bytes, workspace_layout(dc).total);
+  if (s != AB_OK) return s;
   s = do_select(dc, Q, K, P, nullptr, nullptr, workspace, ws_bytes, st);
   if (s != AB_OK) return s;
   s = do_sample(dc, P, idx, pi_q32, count, st, d.H, int64_t(bh0) * d.Nq);
@@ -615,9 +630,9 @@ ab_status ab_forward_host(const ab_params* p, const void* Q_host, const void* K_
   NvtxRange nvtx("ab_forward_host");
   ab_status s = check_params(p, true, &d);
   if (s != AB_OK) return s;
-  if (!Q_host || !K_host || !V_host || !O_host || !Q || !K || !V || !O || !idx || !pi_q32 || !count)
-    return AB_ERR_INVALID_ARG;
-  if (ws_bytes < workspace_layout(d).total) return AB_ERR_WORKSPACE;
+  if (!Q_host || !K_host || !V_host || !O_host) return AB_ERR_INVALID_ARG;
+  s = check_path_args(Q, K, V, P, idx, pi_q32, count, O, workspace, ws_bytes, workspace_layout(d).total);
+  if (s != AB_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t q_head = size_t(d.L) * d.d * 2, kv_head = size_t(d.Lk) * d.d * 2;  // bytes per (b, h)
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;

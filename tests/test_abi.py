@@ -136,3 +136,41 @@ def test_forward_slice_range_checked_on_host(lib):
     for bh0, nbh in ((0, 0), (-1, 2), (5, 2), (0, 7)):
         assert lib.ab_forward_slice(ctypes.byref(p), bh0, nbh, *args) == 1
     assert lib.ab_forward_slice(ctypes.byref(p), 0, 2, good, good, None, *args[3:]) == 1  # V missing
+
+
+def test_select_sample_checked_on_host(lib):
+    # null, misaligned and workspace errors are found before anything is
+    # enqueued, both for rows the fused kernel takes (Nkv <= 2048) and for
+    # longer rows, which run the two launches (pointers never read)
+    good, bad = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1008)
+    for L in (256, 2049 * 16):  # Nkv = 16 and 2049
+        p = ab.Params(B=1, H=1, L=L, d=64, q_block=64, kv_block=16, C=4).c()
+        big = ctypes.c_size_t(1 << 40)
+        assert lib.ab_select_sample(ctypes.byref(p), None, None, None, None, None, None, None, 0, None) == 1
+        assert lib.ab_select_sample(ctypes.byref(p), good, good, good, None, good, good, good, big, None) == 1
+        assert lib.ab_select_sample(ctypes.byref(p), good, good, good, good, good, bad, good, big, None) == 1
+        assert lib.ab_select_sample(ctypes.byref(p), good, good, good, good, good, good, good,
+                                    ctypes.c_size_t(16), None) == 6
+
+
+def test_whole_path_calls_check_every_argument_first(lib):
+    # ab_forward, ab_forward_slice and ab_forward_host find a null or
+    # misaligned buffer (or a short workspace) before anything is enqueued,
+    # whichever buffer it is (pointers never read)
+    p = ab.Params(B=1, H=2, L=256, d=64, q_block=64, kv_block=16, C=4).c()
+    good, bad = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1008)
+    big, small = ctypes.c_size_t(1 << 40), ctypes.c_size_t(16)
+    # Q, K, V, P, idx, pi_q32, count, O, workspace
+    for k in range(9):
+        for wrong in (None, bad):
+            dev = [good] * 9
+            dev[k] = wrong
+            assert lib.ab_forward(ctypes.byref(p), *dev, big, None) == 1, (k, wrong)
+            assert lib.ab_forward_slice(ctypes.byref(p), 0, 1, *dev, big, None) == 1, (k, wrong)
+            host = [good] * 4
+            assert lib.ab_forward_host(ctypes.byref(p), *host, dev[0], dev[1], dev[2], *dev[3:], big, None) == 1
+    dev = [good] * 9
+    assert lib.ab_forward(ctypes.byref(p), *dev, small, None) == 6
+    assert lib.ab_forward_slice(ctypes.byref(p), 1, 1, *dev, small, None) == 6
+    assert lib.ab_forward_host(ctypes.byref(p), None, good, good, good, *dev, big, None) == 1
+    assert lib.ab_forward_host(ctypes.byref(p), good, good, good, good, *dev, small, None) == 6
