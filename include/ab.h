@@ -218,7 +218,8 @@ ab_status ab_attention_dense(const ab_params* p, const void* Q, const void* K, c
  * IBCS estimate is what SIP samples from), so P is read back from L2 rather
  * than after a DRAM round trip.  Longer rows run the two steps as separate
  * launches.  Arguments as for ab_select (P is still written) and ab_sample;
- * errors as for those two calls.  On a B200 the fused launch measured slower
+ * errors as for those two calls, all found before either step is enqueued.
+ * On a B200 the fused launch measured slower
  * than the two launches (its nine warps per scoring CTA sample with fewer
  * rows in flight than the sampler's own grid), so ab_forward keeps the two.
  */
@@ -228,7 +229,8 @@ ab_status ab_select_sample(const ab_params* p, const void* Q, const void* K, flo
 /*
  * The three steps in order on device buffers: ab_select (into P, with
  * centroids/counts not kept), ab_sample, ab_attention.  `workspace` as for
- * ab_select.
+ * ab_select.  Every buffer is checked (non-null, 16-byte aligned, workspace
+ * size) before the first step is enqueued.
  */
 ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const void* V, float* P,
                      int32_t* idx, uint32_t* pi_q32, int32_t* count, void* O, void* workspace,
@@ -247,7 +249,8 @@ ab_status ab_forward(const ab_params* p, const void* Q, const void* K, const voi
  * are bit-identical to the same heads of ab_forward on the whole problem.
  * `workspace` as for ab_select, sized for the slice (ab_workspace_size of
  * the problem with B = 1, H = nbh).  AB_ERR_INVALID_ARG if the range is
- * empty or leaves [0, B * H).
+ * empty or leaves [0, B * H); buffers are checked as for ab_forward, before
+ * anything is enqueued.
  */
 ab_status ab_forward_slice(const ab_params* p, int32_t bh0, int32_t nbh, const void* Q, const void* K,
                            const void* V, float* P, int32_t* idx, uint32_t* pi_q32, int32_t* count, void* O,
