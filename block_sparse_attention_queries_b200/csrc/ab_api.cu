@@ -147,22 +147,69 @@ ab_status launch_status() {
 }
 
 // ---------------------------------------------------------------- launches
+PFN_cuCtxGetCurrent_v4000 ctx_current_fn();
+
+// The selector's second stream, one per CUDA context, created on first use
+// and kept (like the host pipeline's copy streams): the K-block summaries,
+// which only read K, run on it beside the k-means launch, which only reads
+// Q; the scoring launch waits for both.  A call holds the lock from the fork
+// to the join so that calls from several host threads take turns.
+struct SideStream {
+  CUcontext ctx = nullptr;
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex mu;
+};
+std::mutex g_side_mutex;
+std::vector<SideStream*> g_sides;  // never freed
+
+SideStream* side_stream_current_context() {
+  auto get_ctx = ctx_current_fn();
+  if (!get_ctx) return nullptr;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
+  std::lock_guard<std::mutex> lock(g_side_mutex);
+  for (SideStream* x : g_sides)
+    if (x->ctx == ctx) return x;
+  SideStream* x = new SideStream;
+  x->ctx = ctx;
+  if (cudaStreamCreateWithFlags(&x->s, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&x->fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&x->join, cudaEventDisableTiming) != cudaSuccess) {
+    if (x->fork) cudaEventDestroy(x->fork);
+    if (x->s) cudaStreamDestroy(x->s);
+    delete x;
+    return nullptr;
+  }
+  g_sides.push_back(x);
+  return x;
+}
+
 // sip != nullptr: the scoring kernel also runs SIP on its rows (rows of at
-// most kFusedSampleMaxNkv blocks).
+// most kFusedSampleMaxNkv blocks).  overlap: the K-block summaries run on the
+// context's second stream beside k-means (false: everything on `st`).
 template <int D>
 ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, float* cent, int32_t* counts,
-                     uint8_t* ws, cudaStream_t st, const SipArgs* sip = nullptr) {
+                     uint8_t* ws, cudaStream_t st, const SipArgs* sip = nullptr, bool overlap = true) {
   const Workspace w = workspace_layout(d);
   auto* ksum = reinterpret_cast<__nv_bfloat16*>(ws + w.off_ksum);
   auto* cent_ws = reinterpret_cast<__nv_bfloat16*>(ws + w.off_cent);
   auto* cnt_ws = reinterpret_cast<int32_t*>(ws + w.off_cnt);
 
-  // K-block summaries
+  // K-block summaries, on the second stream when there is one
+  SideStream* side = overlap ? side_stream_current_context() : nullptr;
+  std::unique_lock<std::mutex> side_lock;
+  if (side) {
+    side_lock = std::unique_lock<std::mutex>(side->mu);
+    if (cudaEventRecord(side->fork, st) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+      return AB_ERR_CUDA;
+  }
   {
     const int64_t warps = int64_t(d.BH) * d.Nkv;
-    ksum_kernel<D><<<unsigned((warps + 7) / 8), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(K), ksum,
-                                                              d.BH, d.Lk, d.Nkv, d.kv_block);
+    ksum_kernel<D><<<unsigned((warps + 7) / 8), 256, 0, side ? side->s : st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(K), ksum, d.BH, d.Lk, d.Nkv, d.kv_block);
     if (launch_status() != AB_OK) return AB_ERR_CUDA;
+    if (side && cudaEventRecord(side->join, side->s) != cudaSuccess) return AB_ERR_CUDA;
   }
   // k-means per query block
   {
@@ -185,6 +232,7 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* P, floa
     }
     if (s != AB_OK) return s;
   }
+  if (side && cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess) return AB_ERR_CUDA;
   // scores and block mass
   {
     CUtensorMap tmCent, tmKsum;
@@ -277,13 +325,14 @@ ab_status run_attention(const Dims& d, const void* Q, const void* K, const void*
 }
 
 ab_status do_select(const Dims& d, const void* Q, const void* K, float* P, float* cent, int32_t* counts, void* ws,
-                    size_t ws_bytes, cudaStream_t st) {
+                    size_t ws_bytes, cudaStream_t st, bool overlap = true) {
   if (!Q || !K || !P || !ws) return AB_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(P) || !aligned16(ws)) return AB_ERR_INVALID_ARG;
   if ((cent && !aligned16(cent)) || (counts && !aligned16(counts))) return AB_ERR_INVALID_ARG;
   if (ws_bytes < workspace_layout(d).total) return AB_ERR_WORKSPACE;
   auto* w = reinterpret_cast<uint8_t*>(ws);
-  return d.d == 128 ? run_select<128>(d, Q, K, P, cent, counts, w, st) : run_select<64>(d, Q, K, P, cent, counts, w, st);
+  return d.d == 128 ? run_select<128>(d, Q, K, P, cent, counts, w, st, nullptr, overlap)
+                    : run_select<64>(d, Q, K, P, cent, counts, w, st, nullptr, overlap);
 }
 
 // One warp per row (the row's quantised weights in shared memory), for rows
@@ -708,7 +757,7 @@ ab_status ab_select_static(const ab_params* p, const void* Q, const void* K, flo
   void* scratch = static_scratch_current_device();
   if (!scratch) return AB_ERR_CUDA;
   return do_select(d, Q, K, P, centroids, counts, scratch, size_t(AB_SELECT_STATIC_SCRATCH_BYTES),
-                   static_cast<cudaStream_t>(stream));
+                   static_cast<cudaStream_t>(stream), /*overlap=*/false);
 }
 
 ab_status ab_get_device_error(void* stream, int32_t* code) {

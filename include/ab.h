@@ -38,15 +38,19 @@
  *    (Nkv = ceil(Lk / kv_block)); the last block of each kind may be
  *    partial.
  *  - Memory: the caller allocates and owns every buffer (device memory unless a
- *    call says "host"); the library allocates and frees no memory (the
- *    pipelined ab_forward_host creates two copy streams and four events per
- *    CUDA context on its first call and keeps them).
+ *    call says "host"); the library allocates and frees no memory (it creates
+ *    streams and events once per CUDA context and keeps them: two copy
+ *    streams and four events for the pipelined ab_forward_host, one stream
+ *    and two events on which the selecting calls run the K-block summaries
+ *    beside k-means).
  *    Every device pointer must be 16-byte aligned.
  *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  *    Every call only enqueues work on it and returns; results are ready when
- *    the stream reaches them.  The library keeps no state between calls other
- *    than the device error word, the fixed scratch array behind
- *    ab_select_static and ab_forward_host's copy streams.
+ *    the stream reaches them (work on the library's own streams is joined
+ *    back to `stream` by events, which also works under stream capture).
+ *    The library keeps no state between calls other than the device error
+ *    word, the fixed scratch array behind ab_select_static and those
+ *    streams and events.
  *  - Errors: arguments are checked on the host before anything is launched;
  *    a bad argument returns AB_ERR_INVALID_ARG (or AB_ERR_UNSUPPORTED for a
  *    valid but unimplemented size) and enqueues nothing.  AB_ERR_CUDA reports
