@@ -468,6 +468,36 @@ def test_forward_host_equals_device_path(dev, B, H, grid):
     assert torch.equal(Oh, ref.O.cpu())
 
 
+def test_forward_captured_in_cuda_graph(dev):
+    # the whole path captured into a CUDA graph (the selector's side stream
+    # joins the capture through its fork and join events) and replayed gives
+    # the eager call's lists and output bit for bit, replay after replay
+    grid = (2, 16, 16)
+    p = ab.Params(B=1, H=3, L=512, d=128, q_block=128, kv_block=16, C=8, keep_ratio=0.15, seed=17)
+    _, (Q, K, V), _ = _inputs(p, grid, 8, 23, dev)
+    ref = ab.ab_forward(p, Q, K, V)
+    torch.cuda.synchronize()
+    bufs = ab.Buffers(p, dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        ab.ab_forward(p, Q, K, V, bufs)  # first call on this stream outside the capture
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ab.ab_forward(p, Q, K, V, bufs)
+    for _ in range(3):
+        bufs.O.zero_()
+        bufs.count.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        _no_device_error(dev)
+        assert torch.equal(bufs.count, ref.count)
+        assert torch.equal(bufs.idx, ref.idx)
+        assert torch.equal(bufs.O, ref.O)
+
+
 def test_forward_host_repeated_and_from_two_threads(dev):
     # the pipelined host call keeps its copy streams and events per CUDA
     # context: repeated calls, and calls from two host threads at once (each
