@@ -304,7 +304,10 @@ __global__ void __launch_bounds__(128, C <= 8 ? 5 : 3) kmeans_kernel(const __gri
     for (int c = 0; c < C; ++c) {
       const int4 w4 = *reinterpret_cast<const int4*>(wcnt + 4 * c);
       cnt[c] = (w4.x + w4.y) + (w4.z + w4.w);
-      if (own_dim && cnt[c] > 0) mu[c] = __uint_as_float(sv[c]) / float(cnt[c]);
+      // the sum is exact (bf16 values times a 0/1 one-hot, accumulated in
+      // fp32); dividing by the count with the reciprocal instruction (2 ulp)
+      // instead of an IEEE division takes a fifth of the update's time
+      if (own_dim && cnt[c] > 0) mu[c] = __fdividef(__uint_as_float(sv[c]), float(cnt[c]));
     }
   }
 
